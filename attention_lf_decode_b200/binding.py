@@ -1,0 +1,220 @@
+"""Python binding of the C ABI in ``include/lf_decode.h`` (ctypes).
+
+Argument marshalling only: every step of the decode runs in the CUDA kernels
+of ``liblf_decode.so``.  Tensors are torch CUDA tensors (PyTorch provides
+device memory and streams); they are checked for device, dtype, shape and
+contiguity, and their data pointers are passed through.  There is no CPU
+fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblf_decode.so")
+
+LF_OK = 0
+LF_EINVAL = -1
+LF_ENOTINIT = -2
+LF_ECUDA = -3
+LF_EDEVICE = -4
+LF_EUNSUPPORTED = -5
+LF_STATUS_WAIT_TIMEOUT = 1
+LF_STATUS_NO_CANDIDATE = 2
+
+EXPORTS = ("lf_init", "lf_set_stream", "lf_prefill_cache", "lf_decode_step",
+           "lf_decode_attention", "lf_set_split", "lf_get_split", "lf_get_status",
+           "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version")
+
+
+class LFError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {lf_strerror(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblf_decode.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} is missing: build it with `python -m attention_lf_decode_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, VP = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+    sig = {
+        "lf_init": ([ctypes.POINTER(P), I, I, I, I, I, VP], I),
+        "lf_set_stream": ([P, VP], I),
+        "lf_prefill_cache": ([P, VP, VP, I, VP, VP, VP, I], I),
+        "lf_decode_step": ([P, VP, VP, VP, VP, VP, VP, I, I, I, VP, VP], I),
+        "lf_decode_attention": ([P, VP, VP, VP, VP, VP, VP, I, VP], I),
+        "lf_set_split": ([P, I], I),
+        "lf_get_split": ([P, I], I),
+        "lf_get_status": ([P], I),
+        "lf_status_bits": ([P], I),
+        "lf_destroy": ([P], I),
+        "lf_strerror": ([I], ctypes.c_char_p),
+        "lf_version": ([], I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def lf_strerror(code: int) -> str:
+    return load_library().lf_strerror(int(code)).decode()
+
+
+def lf_version() -> int:
+    return load_library().lf_version()
+
+
+def _check(code: int, what: str) -> int:
+    if code < 0:
+        raise LFError(code, what)
+    return code
+
+
+def _ptr(t, dtype, shape, name):
+    """Data pointer of a contiguous CUDA tensor of the given dtype/shape."""
+    import torch
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Handle:
+    """An ``lf_handle`` plus the shape it was created for."""
+
+    def __init__(self, ptr: ctypes.c_void_p, B, Hq, Hkv, D, max_budget):
+        self.ptr = ptr
+        self.B, self.Hq, self.Hkv, self.D, self.max_budget = B, Hq, Hkv, D, max_budget
+
+    def __del__(self):
+        try:
+            if self.ptr:
+                lf_destroy(self)
+        except Exception:
+            pass
+
+
+def lf_init(B: int, Hq: int, Hkv: int, D: int, max_budget: int, stream=None) -> Handle:
+    """Create a handle on the current CUDA device.  ``stream``: a torch
+    stream, a raw cudaStream_t integer, or None for torch's current stream."""
+    import torch
+    lib = load_library()
+    h = ctypes.c_void_p()
+    _check(lib.lf_init(ctypes.byref(h), B, Hq, Hkv, D, max_budget, _stream_ptr(stream)), "lf_init")
+    return Handle(h, B, Hq, Hkv, D, max_budget)
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def lf_set_stream(h: Handle, stream=None) -> None:
+    _check(load_library().lf_set_stream(h.ptr, _stream_ptr(stream)), "lf_set_stream")
+
+
+def lf_set_split(h: Handle, split: int) -> None:
+    _check(load_library().lf_set_split(h.ptr, split), "lf_set_split")
+
+
+def lf_get_split(h: Handle, budget: int) -> int:
+    return _check(load_library().lf_get_split(h.ptr, budget), "lf_get_split")
+
+
+def lf_prefill_cache(h: Handle, k, v, n: int, kcache, vcache, pos, budget: int) -> None:
+    import torch
+    bf = torch.bfloat16
+    cshape = (h.B, h.Hkv, budget, h.D)
+    kp = _ptr(k, bf, (h.B, h.Hkv, n, h.D), "k") if n > 0 else None
+    vp = _ptr(v, bf, (h.B, h.Hkv, n, h.D), "v") if n > 0 else None
+    _check(load_library().lf_prefill_cache(
+        h.ptr, kp, vp, n, _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget), "lf_prefill_cache")
+
+
+def lf_decode_step(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int, sink: int,
+                   window: int, out, evicted_idx) -> None:
+    import torch
+    bf = torch.bfloat16
+    cshape = (h.B, h.Hkv, budget, h.D)
+    _check(load_library().lf_decode_step(
+        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
+        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget, sink, window,
+        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out"),
+        _ptr(evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step")
+
+
+def lf_decode_attention(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int, out) -> None:
+    import torch
+    bf = torch.bfloat16
+    cshape = (h.B, h.Hkv, budget, h.D)
+    _check(load_library().lf_decode_attention(
+        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
+        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention")
+
+
+def lf_get_status(h: Handle) -> int:
+    """LF_OK, or LF_EDEVICE (bits from lf_status_bits); raises on LF_ECUDA."""
+    code = load_library().lf_get_status(h.ptr)
+    if code not in (LF_OK, LF_EDEVICE):
+        raise LFError(code, "lf_get_status")
+    return code
+
+
+def lf_status_bits(h: Handle) -> int:
+    return _check(load_library().lf_status_bits(h.ptr), "lf_status_bits")
+
+
+def lf_destroy(h: Handle) -> None:
+    if h.ptr:
+        code = load_library().lf_destroy(h.ptr)
+        h.ptr = None
+        _check(code, "lf_destroy")
+
+
+# ---------------------------------------------------------------- helpers
+
+def bf16_from_bits(bits, device="cuda"):
+    """torch bf16 tensor on ``device`` from a numpy uint16 bit array."""
+    import numpy as np
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device)
+
+
+def bits_from_bf16(t):
+    """numpy uint16 bits of a bf16 tensor (copied to the host)."""
+    import numpy as np
+    return t.detach().contiguous().view(__import__("torch").int16).cpu().numpy().view(np.uint16)

@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Throughput of the fused LongFlow decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one call of lf_decode_step: attention + score + eviction for a
+whole batch, one kernel launch.  Default workload (the throughput point):
+batch 64, 32 query / 8 KV heads, head_dim 128, bf16 cache, budget 4096,
+sink 4, window 128, full cache, 256 distinct synthetic inputs cycled.  The
+1 GiB KV cache read per step is far larger than L2, so no L2 flush is
+needed between steps.
+
+Rank 0 prints ONE JSON line.  Under torchrun each rank runs its own batch
+(weak scaling, no collective on the data path); time is the max over ranks.
+`--impl reference` times the CPU oracle (the reference arm of this build)
+on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+for _v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+    os.environ.setdefault(_v, "1")  # the CPU oracle runs single-threaded
+
+import numpy as np  # noqa: E402
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused decode steps/s per layer and achieved HBM GB/s vs B200 peak"
+UNIT = "steps/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "attention_lf_decode_b200", "csrc", "lf_decode.cu")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_decode_throughput_b64_n4096.md")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--config", default="throughput")
+    ap.add_argument("--split", type=int, default=0, help="CTAs per row (0 = automatic)")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ bytes
+
+def algorithmic_bytes(cfg, filled: int) -> dict:
+    """Bytes one step must move: the K and V of every filled slot once, plus
+    every write (fp32 output, the new token's K/V row, its position, the
+    evicted index).  q, k_new, v_new and the position table are read too;
+    they are listed apart (under 1%)."""
+    rows = cfg.batch * cfg.hkv
+    kv_read = rows * filled * cfg.head_dim * 2 * 2
+    writes = (cfg.batch * cfg.hq * cfg.head_dim * 4 + rows * cfg.head_dim * 2 * 2 + rows * 4
+              + rows * 4)
+    other_reads = (cfg.batch * cfg.hq * cfg.head_dim * 2 + rows * cfg.head_dim * 2 * 2
+                   + rows * cfg.budget * 4)
+    return {"kv_read": kv_read, "writes": writes, "algorithmic": kv_read + writes,
+            "other_reads": other_reads}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in (KERNEL_SRC, os.path.join(ROOT, "attention_lf_decode_b200", "csrc", "lf_ptx.cuh")):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    try:
+        txt = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.e+]+)", txt)
+    if not m or not t or m.group(1) != kernel_hash():
+        return None
+    return float(t.group(1))
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, enabled: bool = True):
+        self.proc = None
+        self.idx = gpu_index
+        if enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ oracle
+
+def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_steps: int):
+    """Time the CPU oracle, as it stands, on sampled batch entries; returns
+    (full steps/s extrapolated from rows/s, sample description, steps run)."""
+    import oracle
+    from attention_lf_decode_b200 import synth
+    kc, vc, pos = synth.prefill_layout(kpre_bits[batch_sel], vpre_bits[batch_sel], cfg.budget)
+    K, V = synth.bf16_bits_to_f64(kc), synth.bf16_bits_to_f64(vc)
+    P = pos.astype(np.int64)
+    del kc, vc
+    rows = len(batch_sel) * cfg.hkv
+    t_total, n = 0.0, 0
+    while n < max_steps and (t_total < seconds or n == 0):
+        qb, knb, vnb = gen.step_inputs(n)
+        q = synth.bf16_bits_to_f64(qb[batch_sel])
+        kn = synth.bf16_bits_to_f64(knb[batch_sel])
+        vn = synth.bf16_bits_to_f64(vnb[batch_sel])
+        t0 = time.perf_counter()
+        res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window)
+        t_total += time.perf_counter() - t0
+        K, V, P = res.kcache, res.vcache, res.pos
+        n += 1
+    per_row = t_total / (n * rows)
+    full_rows = cfg.batch * cfg.hkv
+    rate = 1.0 / (per_row * full_rows)
+    sample = (f"{n} step(s) on {len(batch_sel)} of {cfg.batch} batch entries "
+              f"({rows} of {full_rows} rows), {t_total:.1f} s; steps/s scaled to all rows")
+    return rate, sample, n
+
+
+def threads_used():
+    v = os.environ.get("OMP_NUM_THREADS") or os.environ.get("OPENBLAS_NUM_THREADS")
+    return int(v) if v and v.isdigit() else os.cpu_count()
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from attention_lf_decode_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    workload = (f"{cfg.name}: batch {cfg.batch}, {cfg.hq} query / {cfg.hkv} KV heads, "
+                f"head_dim {cfg.head_dim}, bf16 KV cache, budget {cfg.budget}, sink {cfg.sink}, "
+                f"window {cfg.window}, prefill {cfg.prefill}")
+
+    if args.impl == "reference":
+        return reference_arm(args, cfg, workload, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    from attention_lf_decode_b200 import binding
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    # per-rank synthetic data: the same recipe, a different seed per rank
+    rcfg = cfg.with_(seed=cfg.seed + 1000 * rank) if rank else cfg
+    gen = synth.SynthDecode(rcfg)
+    t0 = time.time()
+    kpre, vpre = gen.prefill()
+    log(f"[rank {rank}] prefill drawn in {time.time() - t0:.1f} s")
+    n_inputs = min(cfg.steps, 256)
+    inputs = [gen.step_inputs(s) for s in range(n_inputs)]
+
+    stream = torch.cuda.current_stream()
+    h = binding.lf_init(cfg.batch, cfg.hq, cfg.hkv, cfg.head_dim, cfg.budget, stream)
+    if args.split:
+        binding.lf_set_split(h, args.split)
+    split = binding.lf_get_split(h, cfg.budget)
+    dev = "cuda"
+    kcache = torch.empty((cfg.batch, cfg.hkv, cfg.budget, cfg.head_dim), dtype=torch.bfloat16, device=dev)
+    vcache = torch.empty_like(kcache)
+    pos = torch.empty((cfg.batch, cfg.hkv, cfg.budget), dtype=torch.int32, device=dev)
+    binding.lf_prefill_cache(h, binding.bf16_from_bits(kpre), binding.bf16_from_bits(vpre),
+                             cfg.prefill, kcache, vcache, pos, cfg.budget)
+    q_all = torch.stack([binding.bf16_from_bits(x[0]) for x in inputs])
+    kn_all = torch.stack([binding.bf16_from_bits(x[1]) for x in inputs])
+    vn_all = torch.stack([binding.bf16_from_bits(x[2]) for x in inputs])
+    out = torch.empty((cfg.batch, cfg.hq, cfg.head_dim), dtype=torch.float32, device=dev)
+    ev = torch.empty((cfg.batch, cfg.hkv), dtype=torch.int32, device=dev)
+
+    def step(i):
+        j = i % n_inputs
+        binding.lf_decode_step(h, q_all[j], kn_all[j], vn_all[j], kcache, vcache, pos, cfg.budget,
+                               cfg.sink, cfg.window, out, ev)
+
+    # warm-up
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    if binding.lf_get_status(h) != binding.LF_OK:
+        raise RuntimeError(f"device status bits {binding.lf_status_bits(h)} after warm-up")
+
+    # timed region: K back-to-back steps, CUDA events on the launching stream
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank, enabled=not args.no_clocks)
+    time.sleep(0.3 if not args.no_clocks else 0.0)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if binding.lf_get_status(h) != binding.LF_OK:
+        raise RuntimeError(f"device status bits {binding.lf_status_bits(h)} in the timed region")
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+        dist.barrier()
+    ms_per_step = ms_max / args.steps
+    value = world * args.steps / (ms_max / 1e3)
+
+    # end to end: pinned host inputs -> device, step, result -> pinned host, every step
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(np.stack([x[0] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        hk = torch.from_numpy(np.stack([x[1] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        hv = torch.from_numpy(np.stack([x[2] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        d_q = torch.empty_like(q_all[0])
+        d_k = torch.empty_like(kn_all[0])
+        d_v = torch.empty_like(vn_all[0])
+        h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        h_ev = torch.empty(ev.shape, dtype=torch.int32).pin_memory()
+        n_e2e = args.e2e_steps
+
+        def e2e_step(i):
+            j = i % n_inputs
+            d_q.copy_(hq[j], non_blocking=True)
+            d_k.copy_(hk[j], non_blocking=True)
+            d_v.copy_(hv[j], non_blocking=True)
+            binding.lf_decode_step(h, d_q, d_k, d_v, kcache, vcache, pos, cfg.budget, cfg.sink,
+                                   cfg.window, out, ev)
+            h_out.copy_(out, non_blocking=True)
+            h_ev.copy_(ev, non_blocking=True)
+            stream.synchronize()
+            return float(h_out[0, 0, 0])  # the host reads the step's result
+
+        for i in range(3):
+            e2e_step(i)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(n_e2e):
+            e2e_step(i)
+        a1.record(stream)
+        a1.synchronize()
+        ems = a0.elapsed_time(a1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
+        d2h = h_out.numel() * 4 + h_ev.numel() * 4
+        e2e = {"value": world * n_e2e / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": ems / n_e2e,
+               "note": "per step: pinned H2D of q/k_new/v_new, lf_decode_step, D2H of out and "
+                       "evicted_idx, stream sync; the KV cache stays resident"}
+        if binding.lf_get_status(h) != binding.LF_OK:
+            raise RuntimeError("device status after e2e")
+
+    by = algorithmic_bytes(cfg, cfg.budget if cfg.prefill >= cfg.budget else cfg.prefill)
+    kern_s = ms_per_step / 1e3  # one launch per step
+    achieved = by["algorithmic"] / kern_s / 1e9
+    peak, peak_src = measured_peak()
+    traffic = ncu_traffic()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, sample, _ = oracle_rate(cfg, gen, kpre, vpre, args.cpu_seconds, list(range(4)), 64)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
+               "sample": sample}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    binding.lf_destroy(h)
+    if rank != 0:
+        return 0
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": workload, "batch": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv,
+            "head_dim": cfg.head_dim, "budget": cfg.budget, "sink": cfg.sink,
+            "window": cfg.window, "kv_dtype": "bf16", "accumulate": "f32",
+            "parallelism": f"dp{world} (batch per rank, no collective)",
+            "split_ctas_per_row": split,
+            "l2": "inputs larger than L2: each step reads the 1 GiB K/V cache (L2 is 126 MB)",
+            "tokens_per_s": value * cfg.batch,
+            "us_per_step_per_layer": ms_per_step * 1e3,
+            "inputs_cycled": n_inputs,
+        },
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": peak_src,
+                     "bytes_per_launch": by["algorithmic"],
+                     "kernel": "lf::fused_decode_kernel<128,4,true>"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def reference_arm(args, cfg, workload, world, rank):
+    """The CPU oracle as the reference arm: each of the W + K steps is a
+    bounded sample (a few rows of the batch), the value is scaled to full
+    steps/s.  Only rank 0 works under torchrun."""
+    if rank != 0:
+        return 0
+    from attention_lf_decode_b200 import synth
+    import oracle
+    gen = synth.SynthDecode(cfg)
+    sel = [0]  # one batch entry = hkv rows per sample
+    kb, vb = gen.prefill(sel)
+    kc, vc, pos = synth.prefill_layout(kb, vb, cfg.budget)
+    K, V, P = synth.bf16_bits_to_f64(kc), synth.bf16_bits_to_f64(vc), pos.astype(np.int64)
+    budget_s = 150.0
+    rows_full = cfg.batch * cfg.hkv
+    # calibrate: one row-step
+    qb, knb, vnb = gen.step_inputs(0)
+    t0 = time.perf_counter()
+    oracle.decode_step(K[:, :1], V[:, :1], P[:, :1], synth.bf16_bits_to_f64(qb[:1, :cfg.group]),
+                       synth.bf16_bits_to_f64(knb[:1, :1]), synth.bf16_bits_to_f64(vnb[:1, :1]),
+                       cfg.sink, cfg.window)
+    t_row = time.perf_counter() - t0
+    nsteps = args.warmup + args.steps
+    rows_per_step = int(max(1, min(cfg.hkv, budget_s / max(nsteps, 1) / max(t_row, 1e-6))))
+    heads = rows_per_step
+    t_total = 0.0
+    for s in range(nsteps):
+        qb, knb, vnb = gen.step_inputs(s % 256)
+        q = synth.bf16_bits_to_f64(qb[:1, :heads * cfg.group])
+        kn = synth.bf16_bits_to_f64(knb[:1, :heads])
+        vn = synth.bf16_bits_to_f64(vnb[:1, :heads])
+        t0 = time.perf_counter()
+        res = oracle.decode_step(K[:, :heads], V[:, :heads], P[:, :heads], q, kn, vn,
+                                 cfg.sink, cfg.window)
+        dt = time.perf_counter() - t0
+        K[:, :heads], V[:, :heads], P[:, :heads] = res.kcache, res.vcache, res.pos
+        if s >= args.warmup:
+            t_total += dt
+    per_row = t_total / (args.steps * heads)
+    value = 1.0 / (per_row * rows_full)
+    sample = (f"each step: oracle on {heads} of {rows_full} rows (batch entry 0), "
+              f"{args.steps} timed steps after {args.warmup} warm-up; steps/s scaled to all rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": workload, "batch": cfg.batch, "budget": cfg.budget},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

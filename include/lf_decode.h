@@ -1,0 +1,163 @@
+/*
+ * lf_decode.h — C ABI of the B200 (sm_100a) LongFlow fused decode step.
+ *
+ * One decode step over a fixed-budget KV cache, in ONE kernel launch:
+ *   1. single-query GQA attention of the current token over every filled
+ *      cache slot plus the new token itself;
+ *   2. a per-slot importance score taken from that same softmax, with no
+ *      history: the probability of the current query averaged over the G
+ *      query heads of the slot's KV group;
+ *   3. when the cache is full, eviction of the lowest-scoring slot that is
+ *      not protected (the first `sink` slots and the last `window`
+ *      positions are protected; ties go to the lowest slot index), and an
+ *      in-place overwrite of that slot with the new token's K/V/position.
+ *      While a slot is still free (position -1), the new token goes to the
+ *      lowest free slot and nothing is evicted.
+ *
+ * Sources: "LongFlow: Efficient KV Cache Compression for Reasoning Models"
+ * (gist.science summary) §2A "Principios de Diseño" (zero-history,
+ * zero-cost importance estimation), §2B "Derivación de la Métrica de
+ * Importancia" (evict the token whose removal least changes the attention
+ * output, scored from its attention weight), §2C "Implementación de Alto
+ * Rendimiento" (static pre-allocated KV cache; one fused kernel doing
+ * attention, importance estimation and eviction); and the blog page
+ * "Долгая память: Оптимизация кэша для сложных рассуждений", sections
+ * "Оптимизированная Реализация с Объединенными Ядрами" (O and the score
+ * produced in one pass over KV blocks and a mask moved between HBM and
+ * on-chip memory) and "Ограничения Памяти при Моделировании Длинных
+ * Последовательностей" (one token evicted after every attention step).
+ * The exact score, the sink/window protection and the tie-break are fixed
+ * by this library's specification, not by the pages.
+ *
+ * Conventions shared by every call
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *     library never frees, keeps or reallocates it.  Layouts are dense,
+ *     row-major, with no padding:
+ *        q       [B, Hq, D]          bf16
+ *        k_new   [B, Hkv, D]         bf16      v_new  [B, Hkv, D]    bf16
+ *        kcache  [B, Hkv, budget, D] bf16      vcache [B, Hkv, budget, D]
+ *        pos     [B, Hkv, budget]    int32, the token position held by each
+ *                                    slot, -1 = free slot
+ *        out     [B, Hq, D]          fp32
+ *        evicted [B, Hkv]            int32
+ *     Query head h reads KV head h / G, G = Hq / Hkv.
+ *   - q, k_new, v_new, kcache, vcache and out must be 16-byte aligned, pos
+ *     and evicted 4-byte aligned.
+ *   - Calls are asynchronous on the stream given to lf_init (or
+ *     lf_set_stream); arguments are checked on the host before anything is
+ *     enqueued.  A failed check enqueues nothing.
+ *   - Return codes (never exceptions): LF_OK, or one of the negative
+ *     LF_E* codes below; lf_strerror names them.
+ */
+#ifndef LF_DECODE_H
+#define LF_DECODE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LF_OK 0
+#define LF_EINVAL (-1)       /* bad argument: null/misaligned pointer, shape, budget, sink, window */
+#define LF_ENOTINIT (-2)     /* null or destroyed handle */
+#define LF_ECUDA (-3)        /* a CUDA runtime call or kernel launch failed */
+#define LF_EDEVICE (-4)      /* the kernel flagged an error (see lf_status_bits) */
+#define LF_EUNSUPPORTED (-5) /* the current device is not sm_100 or lacks a needed feature */
+
+/* device status bits, as set by the kernels and returned by lf_status_bits */
+#define LF_STATUS_WAIT_TIMEOUT 1  /* a bounded wait on a shared-memory barrier gave up */
+#define LF_STATUS_NO_CANDIDATE 2  /* full cache but no unprotected slot (corrupt pos table) */
+
+#if defined(__GNUC__)
+#define LF_API __attribute__((visibility("default")))
+#else
+#define LF_API
+#endif
+
+typedef struct lf_ctx* lf_handle;
+
+/* Create a handle for one attention layer shape on the CURRENT device.
+ *   B, Hq, Hkv, D: batch, query heads, KV heads (Hq % Hkv == 0, Hq/Hkv <= 8),
+ *   head dimension (64 or 128).  max_budget: largest budget later calls may
+ *   pass.  cuda_stream: a cudaStream_t (NULL = legacy default stream).
+ * Allocates one small device status word (cudaMalloc) and nothing else;
+ * later calls never allocate.  On failure *h is set to NULL. */
+LF_API int lf_init(lf_handle* h, int B, int Hq, int Hkv, int D, int max_budget, void* cuda_stream);
+
+/* Change the stream later calls are enqueued on. */
+LF_API int lf_set_stream(lf_handle h, void* cuda_stream);
+
+/* Write a prompt into an empty cache (the statically pre-allocated cache of
+ * "Implementación de Alto Rendimiento"): k, v [B, Hkv, n, D] go to slots
+ * 0..n-1 of kcache/vcache [B, Hkv, budget, D]; pos[j] = j for j < n and -1
+ * after.  0 <= n <= budget <= max_budget, else LF_EINVAL: compressing a
+ * prompt longer than the budget is outside the method, which targets the
+ * decode phase (summary page §5, "Limitaciones").  k and v may be NULL when
+ * n == 0. */
+LF_API int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, int n,
+                     uint16_t* kcache, uint16_t* vcache, int32_t* pos, int budget);
+
+/* THE fused decode step (one kernel launch).  For every row (b, g):
+ *   t = 1 + max(pos) over filled slots (0 for an empty cache);
+ *   out[b, h] = softmax over {filled slots, new token} of
+ *               (q[b,h] . k) / sqrt(D), applied to the matching v;
+ *   if some slot is free: e = lowest free slot, evicted[b,g] = -1;
+ *   else: score_j = mean over the group's heads of the probability of slot
+ *         j, candidates = { j >= sink and pos[j] < t - window },
+ *         e = candidate of lowest score (lowest j on ties), evicted[b,g] = e;
+ *   then kcache/vcache slot e <- k_new/v_new and pos[e] <- t.
+ * Eviction happens after the attention, so it never changes this step's
+ * out.  Requires 1 <= budget <= max_budget, sink >= 0, window >= 1 and
+ * budget > sink + window (so a full cache with distinct positions always
+ * has a candidate).  Positions in pos must be distinct; the kernel flags
+ * LF_STATUS_NO_CANDIDATE, writes evicted = -2 and leaves the row's cache
+ * unchanged when a full row has no candidate.
+ * Near ties: scores are computed in fp32; when the two lowest candidate
+ * scores of a row are within a relative 1e-4 of each other, the kernel
+ * rescores those candidates in fp64 before choosing. */
+LF_API int lf_decode_step(lf_handle h,
+                   const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                   uint16_t* kcache, uint16_t* vcache, int32_t* pos,
+                   int budget, int sink, int window,
+                   float* out, int32_t* evicted_idx);
+
+/* Plain decode attention over filled slots + the new token: the same
+ * kernel with scoring and eviction compiled out.  Nothing is written but
+ * out.  This is the no-eviction control the fused step is timed against. */
+LF_API int lf_decode_attention(lf_handle h,
+                        const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                        const uint16_t* kcache, const uint16_t* vcache, const int32_t* pos,
+                        int budget, float* out);
+
+/* Tuning: number of CTAs (a thread-block cluster) that split one row's
+ * slots; 0 = automatic.  Must be 0 or a power of two <= 16. */
+LF_API int lf_set_split(lf_handle h, int split);
+
+/* The split the next call with this budget would use (after lf_set_split). */
+LF_API int lf_get_split(lf_handle h, int budget);
+
+/* Synchronise the handle's stream, then read and clear the device status
+ * word.  Returns LF_OK if no kernel flagged an error since the last call,
+ * LF_EDEVICE otherwise (the bits are then available from lf_status_bits),
+ * or LF_ECUDA if the stream reported an error. */
+LF_API int lf_get_status(lf_handle h);
+
+/* Status bits captured by the last lf_get_status (LF_STATUS_* above). */
+LF_API int lf_status_bits(lf_handle h);
+
+/* Free the status word and the handle.  Synchronises the stream first. */
+LF_API int lf_destroy(lf_handle h);
+
+/* Static, NUL-terminated name of a return code. */
+LF_API const char* lf_strerror(int code);
+
+/* Library ABI version, (major << 16) | minor. */
+LF_API int lf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LF_DECODE_H */
