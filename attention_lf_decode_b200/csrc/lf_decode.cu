@@ -107,6 +107,7 @@ struct alignas(16) Small {
   unsigned long long wk1[kWarps], wk2[kWarps];
   double wref[kWarps];
   int wref_slot[kWarps];
+  unsigned long long g_key1;       // row-wide lowest key (local copy)
   int g_t, g_free, g_err, g_refine, g_slot;
 };
 
@@ -591,13 +592,14 @@ __global__ void __launch_bounds__(kThreads) fused_decode_kernel(const Params p) 
       }
       sm.g_refine = refine;
       sm.g_slot = (g1 == kNoKey) ? -1 : int(uint32_t(g1 & 0xffffffffull));
-      sm.key1 = g1;  // own copy only; peers have already read the published value
+      // the published key1/key2 stay untouched: peers may still be reading them
+      sm.g_key1 = g1;
     }
     __syncthreads();
 
     if (sm.g_refine) {  // identical decision in every CTA of the cluster
       // fp64 rescoring of the candidates within the tie band
-      const float s1 = __uint_as_float(uint32_t(sm.key1 >> 32));
+      const float s1 = __uint_as_float(uint32_t(sm.g_key1 >> 32));
       const float thr = s1 * (1.0f + kTieRel);
       float w[G];
 #pragma unroll

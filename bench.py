@@ -214,7 +214,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from attention_lf_decode_b200 import binding
+    from attention_lf_decode_b200 import binding, scaling
 
     torch.cuda.set_device(local_rank)
     if world > 1:
@@ -223,7 +223,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
 
     # per-rank synthetic data: the same recipe, a different seed per rank
-    rcfg = cfg.with_(seed=cfg.seed + 1000 * rank) if rank else cfg
+    rcfg = scaling.rank_config(cfg, rank)
     gen = synth.SynthDecode(rcfg)
     t0 = time.time()
     kpre, vpre = gen.prefill()
@@ -278,14 +278,9 @@ def main():
     ms = e0.elapsed_time(e1)
     if binding.lf_get_status(h) != binding.LF_OK:
         raise RuntimeError(f"device status bits {binding.lf_status_bits(h)} in the timed region")
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-        dist.barrier()
+    ms_max = scaling.max_over_ranks(ms, dev)
     ms_per_step = ms_max / args.steps
-    value = world * args.steps / (ms_max / 1e3)
+    value = scaling.whole_job_rate(world, args.steps, ms_max)
 
     # end to end: pinned host inputs -> device, step, result -> pinned host, every step
     e2e = None
@@ -324,14 +319,10 @@ def main():
             e2e_step(i)
         a1.record(stream)
         a1.synchronize()
-        ems = a0.elapsed_time(a1)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = scaling.max_over_ranks(a0.elapsed_time(a1), dev)
         h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
         d2h = h_out.numel() * 4 + h_ev.numel() * 4
-        e2e = {"value": world * n_e2e / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": scaling.whole_job_rate(world, n_e2e, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": ems / n_e2e,
                "note": "per step: pinned H2D of q/k_new/v_new, lf_decode_step, D2H of out and "
