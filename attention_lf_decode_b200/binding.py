@@ -26,7 +26,8 @@ LF_STATUS_NO_CANDIDATE = 2
 
 EXPORTS = ("lf_init", "lf_set_stream", "lf_prefill_cache", "lf_decode_step",
            "lf_decode_attention", "lf_set_split", "lf_get_split", "lf_get_status",
-           "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version")
+           "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version",
+           "lf_decode_step_noalloc")
 
 
 class LFError(RuntimeError):
@@ -61,6 +62,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lf_destroy": ([P], I),
         "lf_strerror": ([I], ctypes.c_char_p),
         "lf_version": ([], I),
+        "lf_decode_step_noalloc": ([VP, VP, VP, VP, VP, VP, I, I, I, I, I, I, I, VP, VP, VP], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -183,6 +185,26 @@ def lf_decode_attention(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget:
         _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
         _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
         _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention")
+
+
+def lf_decode_step_noalloc(q, k_new, v_new, kcache, vcache, pos, budget: int, sink: int,
+                           window: int, out, evicted_idx, stream=None) -> None:
+    """lf_decode_step without a handle and without any device allocation
+    (for callers that cannot allocate; see include/lf_decode.h).  Shapes are
+    taken from the tensors: q [B, Hq, D], kcache [B, Hkv, budget, D]."""
+    import torch
+    bf = torch.bfloat16
+    B, Hq, D = q.shape
+    Hkv = kcache.shape[1]
+    cshape = (B, Hkv, budget, D)
+    _check(load_library().lf_decode_step_noalloc(
+        _ptr(q, bf, (B, Hq, D), "q"), _ptr(k_new, bf, (B, Hkv, D), "k_new"),
+        _ptr(v_new, bf, (B, Hkv, D), "v_new"), _ptr(kcache, bf, cshape, "kcache"),
+        _ptr(vcache, bf, cshape, "vcache"), _ptr(pos, torch.int32, (B, Hkv, budget), "pos"),
+        B, Hq, Hkv, D, budget, sink, window,
+        _ptr(out, torch.float32, (B, Hq, D), "out"),
+        _ptr(evicted_idx, torch.int32, (B, Hkv), "evicted_idx"), _stream_ptr(stream)),
+        "lf_decode_step_noalloc")
 
 
 def lf_get_status(h: Handle) -> int:

@@ -44,6 +44,7 @@
 #include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -1032,6 +1033,105 @@ int lf_destroy(lf_handle h) {
   h->magic = 0;
   free(h);
   return LF_OK;
+}
+
+// ----------------------------------------------------------------------
+// Allocation-free entry point.  Its scratch (the kernel's status word) is a
+// file-scope device array; host code only ever passes the device address
+// that cudaGetSymbolAddress returns for it, looked up once per device.
+// ----------------------------------------------------------------------
+
+constexpr int kNoAllocScratchBytes = 256;
+constexpr int kNoAllocMaxDevices = 64;
+static __device__ __align__(256) int g_lf_noalloc_scratch[kNoAllocScratchBytes / sizeof(int)];
+
+namespace {
+
+struct NoAllocDevice {
+  bool ready;
+  int* scratch;  // device address of g_lf_noalloc_scratch on this device
+  int sm_count;
+  int smem_optin;
+  int major, minor;
+};
+
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+// Once per device, with that device current.
+int noalloc_setup(int dev, NoAllocDevice** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return LF_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc_dev[dev];
+  if (!d.ready) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_lf_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return LF_ECUDA;
+    int sms = 0, optin = 0, major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return LF_ECUDA;
+    d.scratch = static_cast<int*>(ptr);
+    d.sm_count = sms;
+    d.smem_optin = optin;
+    d.major = major;
+    d.minor = minor;
+    d.ready = true;
+  }
+  *out = &d;
+  return LF_OK;
+}
+
+}  // namespace
+
+int lf_decode_step_noalloc(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                           uint16_t* kcache, uint16_t* vcache, int32_t* pos, int B, int Hq,
+                           int Hkv, int D, int budget, int sink, int window, float* out,
+                           int32_t* evicted_idx, void* cuda_stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return LF_EINVAL;
+  const int G = Hq / Hkv;
+  if (G > lf::kMaxG || (D != 64 && D != 128)) return LF_EINVAL;
+  if (budget < 1 || budget > (1 << 22) || long(B) * Hkv > 65535) return LF_EINVAL;
+  // scratch this call needs: one status word
+  const size_t scratch_needed = sizeof(int);
+  if (scratch_needed > size_t(kNoAllocScratchBytes)) return LF_EINVAL;
+
+  // the argument checks of lf_decode_step, before anything is enqueued
+  if (!q || !k_new || !v_new || !kcache || !vcache || !pos || !out || !evicted_idx)
+    return LF_EINVAL;
+  if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(kcache, 16) ||
+      !aligned(vcache, 16) || !aligned(out, 16) || !aligned(pos, 4) || !aligned(evicted_idx, 4))
+    return LF_EINVAL;
+  if (sink < 0 || window < 1 || budget <= sink + window) return LF_EINVAL;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LF_ECUDA;
+  NoAllocDevice* d = nullptr;
+  const int rc = noalloc_setup(dev, &d);
+  if (rc != LF_OK) return rc;
+  if (d->major != 10 || d->minor != 0) return LF_EUNSUPPORTED;
+
+  lf_ctx c;  // on the stack: nothing is allocated
+  memset(&c, 0, sizeof(c));
+  c.B = B;
+  c.Hq = Hq;
+  c.Hkv = Hkv;
+  c.D = D;
+  c.G = G;
+  c.max_budget = budget;
+  c.stream = static_cast<cudaStream_t>(cuda_stream);
+  c.device = dev;
+  c.sm_count = d->sm_count;
+  c.smem_optin = d->smem_optin;
+  c.split_override = 0;
+  c.status = d->scratch;
+  c.magic = kMagic;
+  // the status word starts at zero for every call
+  if (cudaMemsetAsync(d->scratch, 0, scratch_needed, c.stream) != cudaSuccess) return LF_ECUDA;
+  return run_decode(&c, q, k_new, v_new, kcache, vcache, pos, budget, sink, window, out,
+                    evicted_idx, true);
 }
 
 }  // extern "C"

@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", default="throughput")
     ap.add_argument("--split", type=int, default=0, help="CTAs per row (0 = automatic)")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
@@ -205,6 +206,8 @@ def main():
 
     from attention_lf_decode_b200 import synth
     cfg = synth.CONFIGS[args.config]
+    if args.batch:
+        cfg = cfg.with_(batch=args.batch)
     workload = (f"{cfg.name}: batch {cfg.batch}, {cfg.hq} query / {cfg.hkv} KV heads, "
                 f"head_dim {cfg.head_dim}, bf16 KV cache, budget {cfg.budget}, sink {cfg.sink}, "
                 f"window {cfg.window}, prefill {cfg.prefill}")

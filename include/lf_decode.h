@@ -156,6 +156,37 @@ LF_API const char* lf_strerror(int code);
 /* Library ABI version, (major << 16) | minor. */
 LF_API int lf_version(void);
 
+/* lf_decode_step for callers that cannot allocate device memory.
+ *
+ * The LongFlow pages have no counterpart to this call; it exists for users
+ * of this library.  lf_init allocates the device status word the fused
+ * kernel writes its error bits into, and some callers cannot make that
+ * cudaMalloc: runtimes that reserve the device memory up front in a pool of
+ * their own and forbid allocations outside it, or hosts that hand a kernel
+ * only its buffers and a stream.  This entry point takes no handle and
+ * allocates nothing.  Its scratch, the status word, lives in a fixed
+ * 256-byte array in the library's device memory (a file-scope __device__
+ * array), which every GPU that loads the library holds until the process
+ * exits.  The kernel needs one 4-byte word of it, whatever the sizes; a call
+ * whose scratch would not fit is rejected with LF_EINVAL.
+ *
+ * Arguments, layouts, alignment and results are those of lf_decode_step,
+ * with the shape (B, Hq, Hkv, D) and the stream passed directly (budget is
+ * capped at 1 << 22).  The status word is cleared on the stream before the
+ * launch.  Device-side errors are not reported through lf_get_status: a row
+ * the kernel could not evict shows evicted_idx = -2 and an unchanged cache.
+ *
+ * The first call on a device sets up that device (with it current): it
+ * looks up the device address of the scratch array and the device's limits.
+ * Make that first call before any stream capture.  All calls share the one
+ * scratch array, so calls that overlap on the GPU (on different streams)
+ * race on the status word; results in out, evicted_idx and the cache are
+ * not affected. */
+LF_API int lf_decode_step_noalloc(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                  uint16_t* kcache, uint16_t* vcache, int32_t* pos,
+                                  int B, int Hq, int Hkv, int D, int budget, int sink, int window,
+                                  float* out, int32_t* evicted_idx, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
