@@ -11,32 +11,37 @@
 // and score produced in one pass over KV blocks and a mask streamed from HBM
 // into on-chip memory).
 //
-// Design (one row = one (batch, KV head) pair; its K and V slabs are each
-// [budget, D] bf16, contiguous):
-//   * A thread-block cluster of S CTAs splits the row's slots into S chunks
-//     (flash-decoding split).  Each CTA has 4 consumer warps and 1 producer
-//     warp.
-//   * The producer streams the chunk's K tiles, then its V tiles (8 KB each,
-//     contiguous), with 1-D bulk async copies into a 6-stage shared-memory
-//     ring guarded by mbarriers.  Tiles whose slots are all free are never
-//     loaded.  No multicast: every CTA fetches its own tiles.
-//   * K phase: 8 lanes per slot, 16-byte conflict-free shared loads, fp32
-//     FMAs against the pre-scaled query heads held in registers, then a
-//     reduce-scatter over the 8 lanes.  Logits (log2 domain) stay in shared
-//     memory: the exact normalised probabilities need the row-wide max and
-//     sum, which only exist after every CTA of the cluster is done.
-//   * V phase: p = 2^(s - m_cta) in place, o += p * v with one lane per 4
-//     (D = 128) or 2 (D = 64) dims.
-//   * Cluster exchange through distributed shared memory (no global
-//     scratch, no second launch): row max / sum per head, newest position,
-//     lowest free slot.  Each CTA then scores its own slots (exact
-//     normalised probability averaged over the group's heads), reduces a
-//     packed (fp32 score bits << 32 | slot) key to its two lowest values,
-//     and combines its share of the output from all partial outputs.
+// Design.  One row = one (batch, KV head) pair; its K and V slabs are each
+// [budget, D] bf16, contiguous.
+//   * Persistent thread-block clusters: a cluster of S CTAs owns a row at a
+//     time and splits its slots into S chunks (flash-decoding split); the
+//     cluster then moves on to row + (number of clusters).  Each CTA has 8
+//     consumer warps and 1 producer warp.
+//   * The producer streams the chunk's K tiles, then its V tiles (16 KB each,
+//     contiguous) with 1-D bulk async copies into an mbarrier-guarded ring,
+//     without a pause between rows: while the consumers finish one row, the
+//     next row's position table, query heads and new K/V are already loaded
+//     and its first tiles are in flight.  Tiles whose slots are all free are
+//     never loaded.  No multicast: every CTA fetches its own tiles.
+//   * K phase: 8 lanes per slot, 16-byte conflict-free shared loads, packed
+//     fp32x2 FMAs against the pre-scaled query heads held in registers in a
+//     per-lane head order that lets the 8-lane reduce-scatter run without
+//     selects.  Logits (log2 domain) stay in shared memory: the exact
+//     normalised probabilities need the row-wide max and sum, which only
+//     exist once every CTA of the cluster is done.
+//   * V phase: p = 2^(s - m_cta) in place, o += p * v with 8 dims per lane
+//     and packed FMAs.
+//   * Cluster exchange through distributed shared memory, signalled by
+//     remote mbarrier arrivals (release / acquire at cluster scope) into
+//     per-row-parity buffers, so no whole-cluster barrier stops the
+//     producer: row max / sum per head, newest position, lowest free slot;
+//     then each CTA scores its own slots (exact normalised probability
+//     averaged over the group's heads), reduces packed (fp32 score bits << 32
+//     | slot) keys to the two lowest, and combines its share of the output.
 //   * Near ties (two lowest scores within a relative 1e-4) are rescored in
-//     fp64 from the cache, so the choice matches the exact ranking.
-//   * CTA rank 0 writes k_new / v_new / t into the chosen slot, after a
-//     cluster barrier that follows the last read of that slot.
+//     fp64 from the cache, so the choice follows the exact ranking.
+//   * CTA rank 0 writes k_new / v_new / t into the chosen slot after the key
+//     exchange, which every CTA enters only after its last read of the row.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <limits.h>
@@ -55,17 +60,18 @@ namespace cg = cooperative_groups;
 
 namespace lf {
 
-constexpr int kTileBytes = 8192;
-constexpr int kStages = 6;
-constexpr int kConsumerWarps = 4;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
-constexpr int kWarps = kConsumerWarps + 1;
+constexpr int kTileBytes = 32768;
+constexpr int kCW = 8;                      // consumer warps
+constexpr int kConsumers = kCW * 32;
+constexpr int kThreads = kConsumers + 32;   // + 1 producer warp
+constexpr int kMaxStages = 8;
+constexpr int kMinStages = 3;
 constexpr int kMaxSplit = 16;
 constexpr int kMaxG = 8;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 constexpr float kTieRel = 1e-4f;                   // near-tie band rescored in fp64
 constexpr unsigned long long kNoKey = ~0ull;
+constexpr int kBarConsumers = 1;                   // named barrier of the consumer warps
 
 struct Params {
   const uint16_t* q;
@@ -77,39 +83,96 @@ struct Params {
   float* out;
   int32_t* evicted;
   int* status;
+  int rows;
   int budget;
   int chunk;
   int sink;
   int window;
-  int pos_vec4;
+  int nstages;
+  int pos_bulk;      // position rows may be bulk-copied (16-byte aligned)
   float qscale2;     // log2(e) / sqrt(D)
   double qscale2_64;
 };
 
-// Per-CTA scalars; the fields marked "published" are read by the other CTAs
-// of the cluster through distributed shared memory.
+// Per-CTA values that the other CTAs of the cluster read through
+// distributed shared memory (one copy per row parity).
 template <int GP>
-struct alignas(16) Small {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  unsigned long long key1, key2;  // published: two lowest candidate keys
-  double ref_score;               // published: fp64 rescoring result
-  int ref_slot;                   // published
-  int maxpos;                     // published: newest position in the chunk
-  int first_free;                 // published: lowest free slot (global index)
-  int err;                        // published: a bounded wait gave up
-  float m[GP];                    // published: chunk max logit per head
-  float l[GP];                    // published: chunk sum of 2^(s - m) per head
-  float s_new[GP];                // new token logit per head (log2 domain)
-  float Mg[GP], Lg[GP];           // row max / sum per head
-  float cf[kMaxSplit][GP];        // 2^(m_r - M) per cluster rank and head
-  float wmax[kConsumerWarps][GP];
-  float wsum[kConsumerWarps][GP];
-  unsigned long long wk1[kWarps], wk2[kWarps];
-  double wref[kWarps];
-  int wref_slot[kWarps];
-  unsigned long long g_key1;       // row-wide lowest key (local copy)
+struct Pub {
+  float m[GP];   // chunk max logit per head (log2 domain)
+  float l[GP];   // chunk sum of 2^(s - m) per head
+  int maxpos;    // newest position in the chunk (-1: none)
+  int first_free;
+  int err;
+  int pad0;
+  unsigned long long key1, key2;  // two lowest candidate keys
+  double ref_score;               // fp64 rescoring result
+  int ref_slot;
+  int pad1;
+};
+
+// CTA-local barriers and scalars.
+template <int GP>
+struct Local {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t row_full[2];  // row metadata (positions, q, k_new, v_new) landed
+  uint64_t row_free[2];  // consumers are done with a metadata buffer
+  uint64_t xa[2];        // cluster exchange: max / sum / positions published
+  uint64_t xb[2];        // cluster exchange: candidate keys published
+  uint64_t xc[2];        // cluster exchange: fp64 rescoring published
+  float s_new[GP];
+  float Mg[GP], Lg[GP];
+  float cf[kMaxSplit][GP];
+  float wmax[kCW][GP];
+  float wsum[kCW][GP];
+  int wpmax[kCW], wpfree[kCW];
+  unsigned long long wk1[kCW], wk2[kCW];
+  double wref[kCW];
+  int wrefs[kCW];
+  unsigned long long g_key1;
   int g_t, g_free, g_err, g_refine, g_slot;
+  int err;
+};
+
+__host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
+
+template <int D, int G>
+struct Geometry {
+  static constexpr int T = kTileBytes / (2 * D);   // slots per tile: 64 | 128
+  static constexpr int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
+  static constexpr int CPL = D / 64;               // K phase: 16-byte chunks per lane
+  static constexpr int DPL = CPL * 8;              // K phase: dims per lane
+  static constexpr int GROUPS = T / 4;             // K phase: 4-slot groups per tile
+  static constexpr int GPW = GROUPS / kCW;         // K phase: groups per warp per tile
+  // K phase: groups computed together (more in flight hides latency; the
+  // 8-head variants hold twice the query registers, so they take fewer)
+  static constexpr int KU = GP >= 8 ? 1 : (GPW < 4 ? GPW : 4);
+  static constexpr int VL = D / 8;                 // V phase: lanes per slot (8 dims each)
+  static constexpr int SPV = 32 / VL;              // V phase: slots per warp pass
+  static constexpr int TPW = T / kCW;              // V phase: slots per warp per tile
+  static constexpr int VU = TPW / SPV;             // V phase: slot passes unrolled together
+  static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
+  static constexpr size_t kMetaStride = align128(size_t(G) * D * 2 + 2 * D * 2);
+  static constexpr size_t kPubStride = align128(size_t(G) * D * 4 + sizeof(Pub<GP>));
+  static_assert(GROUPS % kCW == 0 && T % kCW == 0 && TPW % SPV == 0, "tile split");
+
+  struct Layout {
+    size_t ring, pl, pos, red, pp, meta, pub, loc, total;
+  };
+  __host__ __device__ static Layout layout(int chunk, int nst) {
+    Layout L;
+    size_t o = 0;
+    L.ring = o; o = align128(o + size_t(nst) * kTileBytes);
+    L.pl = o;   o = align128(o + size_t(chunk) * GP * 4);
+    L.pos = o;  o = align128(o + size_t(2) * chunk * 4);
+    L.red = o;  o = align128(o + size_t(kCW) * G * D * 4);
+    L.pp = o;   o = align128(o + size_t(kCW) * TPW * GP * 8);
+    L.meta = o; o = align128(o + 2 * kMetaStride);
+    L.pub = o;  o = align128(o + 2 * kPubStride);
+    L.loc = o;  o = align128(o + sizeof(Local<GP>));
+    L.total = o;
+    return L;
+  }
 };
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -141,581 +204,753 @@ __device__ __forceinline__ void top2_merge(unsigned long long& k1, unsigned long
   k1 = lo;
   k2 = hi < s2 ? hi : s2;
 }
-
-// One step of the reduce-scatter over the 8 lanes of a slot: with C partial
-// sums per lane, exchange half of them with the lane across `MASK` so that
-// each lane keeps C/2 sums over twice as many lanes.  With C == 1 it is a
-// plain butterfly step (both lanes end with the same sum).
-template <int C, int MASK>
-__device__ __forceinline__ void rs_step(float (&a)[kMaxG], int sub, int& head_base) {
-  if constexpr (C > 1) {
-    constexpr int H = C / 2;
-    const bool hi = (sub & MASK) != 0;
+__device__ __forceinline__ void top2_warp(unsigned long long& k1, unsigned long long& k2) {
 #pragma unroll
-    for (int i = 0; i < H; ++i) {
-      const float send = hi ? a[i] : a[H + i];
-      const float keep = hi ? a[H + i] : a[i];
-      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, MASK);
-    }
-    if (hi) head_base += H;
+  for (int m = 16; m > 0; m >>= 1) {
+    const unsigned long long o1 = __shfl_xor_sync(0xffffffffu, k1, m);
+    const unsigned long long o2 = __shfl_xor_sync(0xffffffffu, k2, m);
+    top2_merge(k1, k2, o1, o2);
+  }
+}
+
+// Any slot of tile `tile` (chunk-local) filled / every slot filled?  Warp-uniform.
+template <int T>
+__device__ __forceinline__ bool tile_filled(const int* ps, int tile, int nvalid, int lane) {
+  bool any = false;
+#pragma unroll
+  for (int k = 0; k < T / 32; ++k) {
+    const int j = tile * T + k * 32 + lane;
+    any |= (j < nvalid) && (ps[j] >= 0);
+  }
+  return __any_sync(0xffffffffu, any);
+}
+template <int T>
+__device__ __forceinline__ bool tile_full(const int* ps, int tile, int nvalid, int lane) {
+  bool all = true;
+#pragma unroll
+  for (int k = 0; k < T / 32; ++k) {
+    const int j = tile * T + k * 32 + lane;
+    all &= (j < nvalid) && (ps[j] >= 0);
+  }
+  return __all_sync(0xffffffffu, all);
+}
+
+// ---- cluster-scope mbarrier signalling (remote arrive, acquire wait)
+__device__ __forceinline__ uint32_t map_rank(const void* p, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void fence_cluster() {
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+  if (try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (try_wait_cluster(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Signal barrier `bar` (same shared-memory offset in every CTA) of all S CTAs.
+__device__ __forceinline__ void signal_cluster(uint64_t* bar, int S) {
+  fence_cluster();
+  for (int r = 0; r < S; ++r) arrive_remote(map_rank(bar, r));
+}
+
+// One reduce-scatter step over the 8 lanes of a slot.  The lane keeps the
+// first C/2 partial sums and sends the rest; because every lane holds its
+// heads in the order k ^ perm(lane), the partner's second half holds exactly
+// the heads of this lane's first half, so no select is needed.  With C == 1
+// it is a butterfly step.
+template <int C, int MASK>
+__device__ __forceinline__ void rs_step(float (&a)[kMaxG]) {
+  if constexpr (C > 1) {
+#pragma unroll
+    for (int i = 0; i < C / 2; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[C / 2 + i], MASK);
   } else {
     a[0] += __shfl_xor_sync(0xffffffffu, a[0], MASK);
   }
 }
 
-// Any slot of tile `tile` (chunk-local) filled?  Warp-uniform.
-template <int T>
-__device__ __forceinline__ bool tile_filled(const int* pos_s, int tile, int nvalid, int lane) {
-  bool any = false;
-#pragma unroll
-  for (int k = 0; k < T / 32; ++k) {
-    const int j = tile * T + k * 32 + lane;
-    any |= (j < nvalid) && (pos_s[j] >= 0);
-  }
-  return __any_sync(0xffffffffu, any);
-}
-
-template <int D, int G>
-struct Geometry {
-  static constexpr int T = kTileBytes / (2 * D);  // slots per tile
-  static constexpr int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
-  static constexpr int CPL = D / 64;              // 16-byte chunks per lane (K phase)
-  static constexpr int DPL = CPL * 8;             // dims per lane (K phase)
-  static constexpr int GROUPS = T / 4;            // 4-slot groups per tile (K phase)
-  static constexpr int DV = D / 32;               // dims per lane (V phase)
-  static constexpr int TPW = T / kConsumerWarps;  // slots per warp per tile (V phase)
-  static constexpr int RC = GP >= 8 ? GP / 8 : 1; // sums a lane holds after reduce-scatter
-  static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
-  static size_t smem_bytes(int chunk) {
-    return size_t(kStages) * kTileBytes + size_t(chunk) * GP * 4 + size_t(chunk) * 4 +
-           size_t(G) * D * 4 + sizeof(Small<GP>);
-  }
-};
-
 template <int D, int G, bool EVICT>
-__global__ void __launch_bounds__(kThreads) fused_decode_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params p) {
   using Geo = Geometry<D, G>;
   constexpr int T = Geo::T, GP = Geo::GP, CPL = Geo::CPL, DPL = Geo::DPL;
-  constexpr int GROUPS = Geo::GROUPS, DV = Geo::DV, TPW = Geo::TPW, RC = Geo::RC;
+  constexpr int GPW = Geo::GPW, KU = Geo::KU, VU = Geo::VU, VL = Geo::VL, SPV = Geo::SPV,
+                TPW = Geo::TPW;
   static_assert(G >= 1 && G <= kMaxG, "group size");
   static_assert(D == 64 || D == 128, "head dim");
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int S = static_cast<int>(cluster.num_blocks());
-  const int row = blockIdx.y;
+  const int ncl = static_cast<int>(gridDim.y), cid = static_cast<int>(blockIdx.y);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int N = p.budget, chunk = p.chunk;
+  const int N = p.budget, chunk = p.chunk, nst = p.nstages;
   const int slot0 = rank * chunk;
   const int nvalid = max(0, min(chunk, N - slot0));
   const int ntiles = (nvalid + T - 1) / T;
+  const int niter = cid < p.rows ? (p.rows - cid + ncl - 1) / ncl : 0;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* ring = smem;
-  float* pl = reinterpret_cast<float*>(ring + kStages * kTileBytes);  // [chunk][GP]
-  int* pos_s = reinterpret_cast<int*>(pl + size_t(chunk) * GP);        // [chunk]
-  float* xo = reinterpret_cast<float*>(pos_s + chunk);                 // [G][D], published
-  Small<GP>& sm = *reinterpret_cast<Small<GP>*>(xo + G * D);
+  const typename Geo::Layout L = Geo::layout(chunk, nst);
+  unsigned char* ring = smem + L.ring;
+  float* pl = reinterpret_cast<float*>(smem + L.pl);     // [chunk][GP] logits, then p
+  int* pos0 = reinterpret_cast<int*>(smem + L.pos);      // [2][chunk]
+  float* red = reinterpret_cast<float*>(smem + L.red);   // [kCW][G][D]
+  float2* pp = reinterpret_cast<float2*>(smem + L.pp);   // [kCW][TPW][GP] (p, p) pairs
+  unsigned char* meta0 = smem + L.meta;                  // [2] {q[G][D], k_new[D], v_new[D]}
+  unsigned char* pub0 = smem + L.pub;                    // [2] {xo[G][D], Pub}
+  Local<GP>& loc = *reinterpret_cast<Local<GP>*>(smem + L.loc);
 
-  // ---------------------------------------------------------------- setup
-  if (tid == 0) {
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kConsumerWarps);
+  // Bounded waits.  After a first wait has given up (error flagged), later
+  // waits only poll once, so a failed launch ends quickly instead of waiting
+  // the full limit at every barrier.
+  auto wait_cta = [&](uint64_t* bar, uint32_t par) {
+    if (*reinterpret_cast<volatile int*>(&loc.err)) {
+      (void)mbar_try_wait(bar, par);
+      return;
     }
-    sm.maxpos = -1;
-    sm.first_free = INT_MAX;
-    sm.err = 0;
+    if (!mbar_wait_bounded(bar, par, kWaitLimitNs)) flag_error(&loc.err, p.status);
+  };
+  auto wait_cl = [&](uint64_t* bar, uint32_t par) {
+    if (*reinterpret_cast<volatile int*>(&loc.err)) {
+      (void)try_wait_cluster(bar, par);
+      return;
+    }
+    if (!wait_cluster_bounded(bar, par)) flag_error(&loc.err, p.status);
+  };
+  auto pos_buf = [&](int b) { return pos0 + b * chunk; };
+  auto q_buf = [&](int b) { return reinterpret_cast<uint16_t*>(meta0 + b * Geo::kMetaStride); };
+  auto kn_buf = [&](int b) { return q_buf(b) + G * D; };
+  auto vn_buf = [&](int b) { return q_buf(b) + G * D + D; };
+  auto xo_buf = [&](int b) { return reinterpret_cast<float*>(pub0 + b * Geo::kPubStride); };
+  auto pub_buf = [&](int b) {
+    return reinterpret_cast<Pub<GP>*>(pub0 + b * Geo::kPubStride + size_t(G) * D * 4);
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < nst; ++s) {
+      mbar_init(&loc.full[s], 1);
+      mbar_init(&loc.empty[s], kCW);
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&loc.row_full[b], 1);
+      mbar_init(&loc.row_free[b], 1);
+      mbar_init(&loc.xa[b], S);
+      mbar_init(&loc.xb[b], S);
+      mbar_init(&loc.xc[b], S);
+    }
+    loc.err = 0;
     fence_mbar_init();
   }
   __syncthreads();
+  cluster.sync();  // every CTA's barriers exist before the first remote arrival
 
-  {  // position table of the chunk -> shared; newest position, lowest free slot
-    int lmax = -1, lfree = INT_MAX;
-    const int32_t* prow = p.pos + size_t(row) * N + slot0;
-    const int nv4 = p.pos_vec4 ? (nvalid >> 2) : 0;
-    for (int i = tid; i < nv4; i += kThreads) {
-      const int4 v = reinterpret_cast<const int4*>(prow)[i];
-      reinterpret_cast<int4*>(pos_s)[i] = v;
-      const int vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (vv[k] >= 0) lmax = max(lmax, vv[k]);
-        else lfree = min(lfree, 4 * i + k);
+  // ring position: tiles issued (producer) or consumed (consumers) so far, and
+  // the stage / phase parity of the next one; both sides walk the same sequence
+  int seq = 0, stg = 0;
+  uint32_t sph = 0;
+
+  if (warp == kCW) {
+    // ================================================================ producer
+    auto issue_meta = [&](int it) {
+      const int row = cid + it * ncl;
+      const int b = it & 1;
+      if (it >= 2 && lane == 0) wait_cta(&loc.row_free[b], uint32_t((it >> 1) & 1) ^ 1u);
+      __syncwarp();
+      int* ps = pos_buf(b);
+      const int32_t* pg = p.pos + size_t(row) * N + slot0;
+      const uint32_t mbytes = uint32_t(G * D * 2 + 2 * D * 2);
+      if (!p.pos_bulk) {
+        for (int j = lane; j < nvalid; j += 32) ps[j] = pg[j];
+        __syncwarp();
+        __threadfence_block();
       }
-    }
-    for (int i = nv4 * 4 + tid; i < nvalid; i += kThreads) {
-      const int v = prow[i];
-      pos_s[i] = v;
-      if (v >= 0) lmax = max(lmax, v);
-      else lfree = min(lfree, i);
-    }
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) {
-      lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, m));
-      lfree = min(lfree, __shfl_xor_sync(0xffffffffu, lfree, m));
-    }
-    if (lane == 0) {
-      if (lmax >= 0) atomicMax(&sm.maxpos, lmax);
-      if (lfree != INT_MAX) atomicMin(&sm.first_free, slot0 + lfree);
-    }
-  }
-
-  const uint16_t* qrow = p.q + size_t(row) * G * D;  // the G query heads of this KV head
-  if (warp == 0) {  // logit of the new token, per head
-    const uint16_t* kn = p.k_new + size_t(row) * D;
-#pragma unroll
-    for (int i = 0; i < G; ++i) {
-      float a = 0.f;
-#pragma unroll
-      for (int d = 0; d < DV; ++d) {
-        const int dd = lane * DV + d;
-        a = fmaf(__uint_as_float(uint32_t(qrow[i * D + dd]) << 16),
-                 __uint_as_float(uint32_t(kn[dd]) << 16), a);
+      if (lane == 0) {
+        const uint32_t pbytes = p.pos_bulk ? uint32_t(nvalid) * 4 : 0u;
+        mbar_arrive_expect_tx(&loc.row_full[b], mbytes + pbytes);
+        if (pbytes) bulk_copy_g2s(ps, pg, pbytes, &loc.row_full[b]);
+        bulk_copy_g2s(q_buf(b), p.q + size_t(row) * G * D, G * D * 2, &loc.row_full[b]);
+        bulk_copy_g2s(kn_buf(b), p.k_new + size_t(row) * D, D * 2, &loc.row_full[b]);
+        bulk_copy_g2s(vn_buf(b), p.v_new + size_t(row) * D, D * 2, &loc.row_full[b]);
       }
-#pragma unroll
-      for (int m = 16; m > 0; m >>= 1) a += __shfl_xor_sync(0xffffffffu, a, m);
-      if (lane == 0) sm.s_new[i] = a * p.qscale2;
-    }
-  }
-  __syncthreads();
-
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    int seq = 0;
-    for (int phase = 0; phase < 2; ++phase) {
-      const uint16_t* base = (phase == 0 ? p.kcache : p.vcache) + (size_t(row) * N + slot0) * D;
+      __syncwarp();
+    };
+    auto issue_tiles = [&](int it, int phase) {
+      const int row = cid + it * ncl;
+      const int* ps = pos_buf(it & 1);
+      const uint16_t* base =
+          (phase == 0 ? p.kcache : p.vcache) + (size_t(row) * N + slot0) * D;
       for (int tile = 0; tile < ntiles; ++tile) {
-        if (!tile_filled<T>(pos_s, tile, nvalid, lane)) continue;
-        const int s = seq % kStages;
-        const uint32_t par = uint32_t(seq / kStages) & 1u;
+        if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
+        const int s = stg;
+        const uint32_t par = sph;
         if (lane == 0) {
-          if (seq >= kStages && !mbar_wait_bounded(&sm.empty[s], par ^ 1u, kWaitLimitNs))
-            flag_error(&sm.err, p.status);
+          if (seq >= nst) wait_cta(&loc.empty[s], par ^ 1u);
           const int ns = min(T, nvalid - tile * T);
           const uint32_t bytes = uint32_t(ns) * D * 2;
-          mbar_arrive_expect_tx(&sm.full[s], bytes);
-          bulk_copy_g2s(ring + s * kTileBytes, base + size_t(tile) * T * D, bytes, &sm.full[s]);
+          mbar_arrive_expect_tx(&loc.full[s], bytes);
+          bulk_copy_g2s(ring + size_t(s) * kTileBytes, base + size_t(tile) * T * D, bytes,
+                        &loc.full[s]);
         }
         __syncwarp();
         ++seq;
+        if (++stg == nst) {
+          stg = 0;
+          sph ^= 1u;
+        }
       }
+    };
+    if (niter > 0) issue_meta(0);
+    for (int it = 0; it < niter; ++it) {
+      wait_cta(&loc.row_full[it & 1], uint32_t((it >> 1) & 1));
+      issue_tiles(it, 0);
+      if (it + 1 < niter) issue_meta(it + 1);
+      issue_tiles(it, 1);
     }
   } else {
-    // ------------------------------------------------------------ consumers
+    // ================================================================ consumers
     const int sub = lane & 7;   // lane within the slot's 8 lanes (K phase)
     const int sig = lane >> 3;  // slot within the warp's 4-slot group (K phase)
+    const int perm = GP >= 8 ? sub : GP == 4 ? ((sub >> 1) & 3) : GP == 2 ? ((sub >> 2) & 1) : 0;
+    const int my_head = perm;   // head whose logit this lane holds after the reduction
+    const bool kwriter = ((sub & Geo::BFLY) == 0) && (my_head < G);
+    const int vsub = lane % VL, vslot = lane / VL;
+    const int eh = lane % GP;   // head of this lane in the probability pass
+    uint32_t xc_uses0 = 0, xc_uses1 = 0;
 
-    float qf[G][DPL];  // query heads, pre-scaled to the log2 domain
+    for (int it = 0; it < niter; ++it) {
+      const int row = cid + it * ncl;
+      const int b = it & 1;
+      const uint32_t bpar = uint32_t((it >> 1) & 1);
+      const int* ps = pos_buf(b);
+      wait_cta(&loc.row_full[b], bpar);
+
+      // query heads of the group, fp32, pre-scaled, in this lane's head order
+      float2 qp[GP][DPL / 2];
+      {
+        const uint16_t* qs = q_buf(b);
 #pragma unroll
-    for (int i = 0; i < G; ++i) {
+        for (int k = 0; k < GP; ++k) {
+          const int h = k ^ perm;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4*>(qrow + i * D + c * 64 + sub * 8);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          for (int c = 0; c < CPL; ++c) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (h < G) w = *reinterpret_cast<const uint4*>(qs + h * D + c * 64 + sub * 8);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          qf[i][c * 8 + 2 * k] = bf16lo(ww[k]) * p.qscale2;
-          qf[i][c * 8 + 2 * k + 1] = bf16hi(ww[k]) * p.qscale2;
+            for (int m = 0; m < 4; ++m)
+              qp[k][c * 4 + m] = make_float2(bf16lo(ww[m]) * p.qscale2, bf16hi(ww[m]) * p.qscale2);
+          }
         }
       }
-    }
+      if (warp == 0) {  // logit of the new token, per head
+        constexpr int DV = D / 32;
+        const uint16_t* qs = q_buf(b);
+        const uint16_t* kn = kn_buf(b);
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          float a = 0.f;
+#pragma unroll
+          for (int d = 0; d < DV; ++d) {
+            const int dd = lane * DV + d;
+            a = fmaf(__uint_as_float(uint32_t(qs[i * D + dd]) << 16),
+                     __uint_as_float(uint32_t(kn[dd]) << 16), a);
+          }
+#pragma unroll
+          for (int m = 16; m > 0; m >>= 1) a += __shfl_xor_sync(0xffffffffu, a, m);
+          if (lane == 0) loc.s_new[i] = a * p.qscale2;
+        }
+      }
+      {  // newest position and lowest free slot of the chunk
+        int mx = -1, fr = INT_MAX;
+        for (int j = tid; j < nvalid; j += kConsumers) {
+          const int v = ps[j];
+          if (v >= 0) mx = max(mx, v);
+          else fr = min(fr, j);
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+          fr = min(fr, __shfl_xor_sync(0xffffffffu, fr, m));
+        }
+        if (lane == 0) {
+          loc.wpmax[warp] = mx;
+          loc.wpfree[warp] = fr == INT_MAX ? INT_MAX : slot0 + fr;
+        }
+      }
+      named_barrier(kBarConsumers, kConsumers);
+      bool fastrow = true;  // every slot of the chunk filled: no per-slot masking
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) fastrow &= (loc.wpfree[w] == INT_MAX);
 
-    int head_base_lane = 0;  // first head whose sums this lane holds
-    float rmax[RC];
+      // ---------------------------------------------------------- K phase
+      float rmax = -INFINITY;
+      for (int tile = 0; tile < ntiles; ++tile) {
+        bool tfull = fastrow && (tile + 1) * T <= nvalid;
+        if (!fastrow) {
+          if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
+          tfull = tile_full<T>(ps, tile, nvalid, lane);
+        }
+        wait_cta(&loc.full[stg], sph);
+        const unsigned char* kt = ring + size_t(stg) * kTileBytes;
+#pragma unroll 1
+        for (int gb = 0; gb < GPW; gb += KU) {
+          float xs[KU];
 #pragma unroll
-    for (int k = 0; k < RC; ++k) rmax[k] = -INFINITY;
-    const bool writer = (sub & Geo::BFLY) == 0;
-
-    // K phase: logits of every filled slot of the chunk
-    int seq = 0;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      if (!tile_filled<T>(pos_s, tile, nvalid, lane)) continue;
-      const int s = seq % kStages;
-      const uint32_t par = uint32_t(seq / kStages) & 1u;
-      if (!mbar_wait_bounded(&sm.full[s], par, kWaitLimitNs)) flag_error(&sm.err, p.status);
-      const unsigned char* kt = ring + s * kTileBytes;
-      const int ns = min(T, nvalid - tile * T);
+          for (int gu = 0; gu < KU; ++gu) {
+            const int si = (warp + (gb + gu) * kCW) * 4 + sig;
+            float2 acc[GP];
 #pragma unroll
-      for (int grp = warp; grp < GROUPS; grp += kConsumerWarps) {
-        const int si = grp * 4 + sig;
-        float a[kMaxG];
+            for (int k = 0; k < GP; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < kMaxG; ++i) a[i] = 0.f;
+            for (int c = 0; c < CPL; ++c) {
+              const uint4 w =
+                  *reinterpret_cast<const uint4*>(kt + si * (2 * D) + c * 128 + sub * 16);
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(kt + si * (2 * D) + c * 128 + sub * 16);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+              for (int m = 0; m < 4; ++m) {
+                const float2 kv = make_float2(bf16lo(ww[m]), bf16hi(ww[m]));
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float k0 = bf16lo(ww[k]), k1 = bf16hi(ww[k]);
+                for (int k = 0; k < GP; ++k) acc[k] = __ffma2_rn(qp[k][c * 4 + m], kv, acc[k]);
+              }
+            }
+            float a[kMaxG];
 #pragma unroll
-            for (int i = 0; i < G; ++i) {
-              a[i] = fmaf(qf[i][c * 8 + 2 * k], k0, a[i]);
-              a[i] = fmaf(qf[i][c * 8 + 2 * k + 1], k1, a[i]);
+            for (int k = 0; k < GP; ++k) a[k] = acc[k].x + acc[k].y;
+            rs_step<GP, 4>(a);
+            rs_step<(GP > 1 ? GP / 2 : 1), 2>(a);
+            rs_step<(GP > 2 ? GP / 4 : 1), 1>(a);
+            xs[gu] = a[0];
+          }
+          if (!tfull) {  // mask free and out-of-range slots
+            const int ns = min(T, nvalid - tile * T);
+#pragma unroll
+            for (int gu = 0; gu < KU; ++gu) {
+              const int si = (warp + (gb + gu) * kCW) * 4 + sig;
+              if (!((si < ns) && (ps[tile * T + si] >= 0))) xs[gu] = -INFINITY;
             }
           }
-        }
-        int hb = 0;
-        rs_step<GP, 4>(a, sub, hb);
-        rs_step<(GP > 1 ? GP / 2 : 1), 2>(a, sub, hb);
-        rs_step<(GP > 2 ? GP / 4 : 1), 1>(a, sub, hb);
-        head_base_lane = hb;
-        const int j = tile * T + si;
-        const bool valid = (si < ns) && (pos_s[j] >= 0);
 #pragma unroll
-        for (int k = 0; k < RC; ++k) {
-          const int h = hb + k;
-          const float x = valid ? a[k] : -INFINITY;
-          if (h < G) {
-            if (writer) pl[j * GP + h] = x;
-            rmax[k] = fmaxf(rmax[k], x);
+          for (int gu = 0; gu < KU; ++gu) {
+            const int j = tile * T + (warp + (gb + gu) * kCW) * 4 + sig;
+            if (kwriter) pl[j * GP + my_head] = xs[gu];
+            rmax = fmaxf(rmax, xs[gu]);
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&loc.empty[stg]);
+        ++seq;
+        if (++stg == nst) {
+          stg = 0;
+          sph ^= 1u;
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[s]);
-      ++seq;
-    }
+      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 8));
+      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 16));
+      if (sig == 0 && kwriter) loc.wmax[warp][my_head] = rmax;
+      named_barrier(kBarConsumers, kConsumers);
 
-    // chunk max per head
-    if (ntiles == 0) {  // no K tile processed: still define the lane's heads
-      int hb = 0;
-      if (GP >= 2 && (sub & 4)) hb += GP / 2;
-      if (GP >= 4 && (sub & 2)) hb += GP / 4;
-      if (GP >= 8 && (sub & 1)) hb += GP / 8;
-      head_base_lane = hb;
-    }
+      float my_m = -INFINITY;
+      if (eh < G) {
 #pragma unroll
-    for (int k = 0; k < RC; ++k) {
-      rmax[k] = fmaxf(rmax[k], __shfl_xor_sync(0xffffffffu, rmax[k], 8));
-      rmax[k] = fmaxf(rmax[k], __shfl_xor_sync(0xffffffffu, rmax[k], 16));
-      const int h = head_base_lane + k;
-      if (sig == 0 && writer && h < G) sm.wmax[warp][h] = rmax[k];
-    }
-    named_barrier(1, kConsumers);
+        for (int w = 0; w < kCW; ++w) my_m = fmaxf(my_m, loc.wmax[w][eh]);
+      }
 
-    const int my_h = lane % GP;  // head of this lane in the probability pass
-    float my_m = -INFINITY;
-    if (my_h < G) {
+      // ---------------------------------------------------------- V phase
+      float2 o[G][4];
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) my_m = fmaxf(my_m, sm.wmax[w][my_h]);
-    }
-
-    // V phase: p = 2^(s - m) in place, o += p v
-    float o[G][DV];
+      for (int i = 0; i < G; ++i)
 #pragma unroll
-    for (int i = 0; i < G; ++i)
+        for (int m = 0; m < 4; ++m) o[i][m] = make_float2(0.f, 0.f);
+      float lsum = 0.f;
+      float2* ppw = pp + warp * TPW * GP;
+      for (int tile = 0; tile < ntiles; ++tile) {
+        bool tfull = fastrow && (tile + 1) * T <= nvalid;
+        if (!fastrow) {
+          if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
+          tfull = tile_full<T>(ps, tile, nvalid, lane);
+        }
+        wait_cta(&loc.full[stg], sph);
+        const unsigned char* vt = ring + size_t(stg) * kTileBytes;
+        // probabilities of this warp's slots, kept for the scores and paired for the FMAs
 #pragma unroll
-      for (int d = 0; d < DV; ++d) o[i][d] = 0.f;
-    float lsum = 0.f;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      if (!tile_filled<T>(pos_s, tile, nvalid, lane)) continue;
-      const int s = seq % kStages;
-      const uint32_t par = uint32_t(seq / kStages) & 1u;
-      if (!mbar_wait_bounded(&sm.full[s], par, kWaitLimitNs)) flag_error(&sm.err, p.status);
-      const unsigned char* vt = ring + s * kTileBytes;
-      const int ns = min(T, nvalid - tile * T);
-#pragma unroll
-      for (int idx = lane; idx < TPW * GP; idx += 32) {
-        const int j = tile * T + warp * TPW + idx / GP;
-        if (my_h < G) {
-          const float x = pl[j * GP + my_h];
-          const float pv = (x == -INFINITY) ? 0.f : exp2f(x - my_m);
-          pl[j * GP + my_h] = pv;
+        for (int idx = lane; idx < TPW * GP; idx += 32) {
+          const int j = tile * T + warp * TPW + idx / GP;
+          float pv = 0.f;
+          if (eh < G) {
+            const float x = pl[j * GP + eh];
+            pv = (x == -INFINITY) ? 0.f : exp2f(x - my_m);
+            pl[j * GP + eh] = pv;
+          }
           lsum += pv;
+          ppw[idx] = make_float2(pv, pv);
+        }
+        __syncwarp();
+        const int ns = tfull ? T : min(T, nvalid - tile * T);
+#pragma unroll VU
+        for (int u = 0; u < TPW / SPV; ++u) {
+          const int ls = u * SPV + vslot;
+          const int si = warp * TPW + ls;
+          const uint4 w = *reinterpret_cast<const uint4*>(vt + si * (2 * D) + vsub * 16);
+          float2 v[4] = {make_float2(bf16lo(w.x), bf16hi(w.x)), make_float2(bf16lo(w.y), bf16hi(w.y)),
+                         make_float2(bf16lo(w.z), bf16hi(w.z)), make_float2(bf16lo(w.w), bf16hi(w.w))};
+          if (!tfull) {  // a free or out-of-range slot may hold anything: keep it out
+            const bool valid = (si < ns) && (ps[tile * T + si] >= 0);
+            if (!valid) {
+#pragma unroll
+              for (int m = 0; m < 4; ++m) v[m] = make_float2(0.f, 0.f);
+            }
+          }
+          const float2* pr = ppw + ls * GP;
+          float2 pi[GP];
+          if constexpr (GP >= 2) {
+#pragma unroll
+            for (int h2 = 0; h2 < GP; h2 += 2) {
+              const float4 f = *reinterpret_cast<const float4*>(pr + h2);
+              pi[h2] = make_float2(f.x, f.y);
+              pi[h2 + 1] = make_float2(f.z, f.w);
+            }
+          } else {
+            pi[0] = pr[0];
+          }
+#pragma unroll
+          for (int i = 0; i < G; ++i)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) o[i][m] = __ffma2_rn(pi[i], v[m], o[i][m]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&loc.empty[stg]);
+        ++seq;
+        if (++stg == nst) {
+          stg = 0;
+          sph ^= 1u;
         }
       }
-      __syncwarp();
-#pragma unroll 4
-      for (int u = 0; u < TPW; ++u) {
-        const int si = warp * TPW + u;
-        const int j = tile * T + si;
-        if (si >= ns || pos_s[j] < 0) continue;  // warp-uniform
-        float pv[GP];
-        if constexpr (GP >= 4) {
+
+      // ---------------------------------------------------- chunk results
 #pragma unroll
-          for (int h4 = 0; h4 < GP; h4 += 4) {
-            const float4 f = *reinterpret_cast<const float4*>(pl + j * GP + h4);
-            pv[h4] = f.x; pv[h4 + 1] = f.y; pv[h4 + 2] = f.z; pv[h4 + 3] = f.w;
-          }
-        } else if constexpr (GP == 2) {
-          const float2 f = *reinterpret_cast<const float2*>(pl + j * GP);
-          pv[0] = f.x; pv[1] = f.y;
-        } else {
-          pv[0] = pl[j];
-        }
-        float vf[DV];
-        if constexpr (DV == 4) {
-          const uint2 w = *reinterpret_cast<const uint2*>(vt + si * (2 * D) + lane * 8);
-          vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
-        } else {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(vt + si * (2 * D) + lane * 4);
-          vf[0] = bf16lo(w); vf[1] = bf16hi(w);
-        }
+      for (int m = GP; m < 32; m <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
+      if (lane < G) loc.wsum[warp][lane] = lsum;
+#pragma unroll
+      for (int msk = VL; msk < 32; msk <<= 1)
 #pragma unroll
         for (int i = 0; i < G; ++i)
 #pragma unroll
-          for (int d = 0; d < DV; ++d) o[i][d] = fmaf(pv[i], vf[d], o[i][d]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[s]);
-      ++seq;
-    }
-
-    // chunk sums per head
+          for (int m = 0; m < 4; ++m) {
+            o[i][m].x += __shfl_xor_sync(0xffffffffu, o[i][m].x, msk);
+            o[i][m].y += __shfl_xor_sync(0xffffffffu, o[i][m].y, msk);
+          }
+      if (vslot == 0) {
 #pragma unroll
-    for (int m = GP; m < 32; m <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
-    if (lane < G) sm.wsum[warp][lane] = lsum;
-
-    // partial outputs of the 4 warps -> xo (the ring is free: all tiles consumed)
-    named_barrier(1, kConsumers);
-    float* red = reinterpret_cast<float*>(ring);  // [warp][G][D]
-#pragma unroll
-    for (int i = 0; i < G; ++i)
-#pragma unroll
-      for (int d = 0; d < DV; ++d) red[(warp * G + i) * D + lane * DV + d] = o[i][d];
-    named_barrier(1, kConsumers);
-    for (int e = tid; e < G * D; e += kConsumers) {
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) acc += red[w * G * D + e];
-      xo[e] = acc;
-    }
-    if (tid < G) {
-      float mm = -INFINITY, ll = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        mm = fmaxf(mm, sm.wmax[w][tid]);
-        ll += sm.wsum[w][tid];
-      }
-      sm.m[tid] = mm;
-      sm.l[tid] = ll;
-    }
-  }
-  __syncthreads();
-
-  // -------------------------------------------- cluster exchange: max / sum
-  cluster.sync();
-  if (tid < G) {
-    const int i = tid;
-    float M = sm.s_new[i];
-    for (int r = 0; r < S; ++r) M = fmaxf(M, cluster.map_shared_rank(&sm, r)->m[i]);
-    float L = exp2f(sm.s_new[i] - M);
-    for (int r = 0; r < S; ++r) {
-      const Small<GP>* pr = cluster.map_shared_rank(&sm, r);
-      const float cf = exp2f(pr->m[i] - M);  // 0 for an empty chunk (m = -inf)
-      sm.cf[r][i] = cf;
-      L += pr->l[i] * cf;
-    }
-    sm.Mg[i] = M;
-    sm.Lg[i] = L;
-  } else if (tid == 32) {
-    int mx = -1, fr = INT_MAX, er = 0;
-    for (int r = 0; r < S; ++r) {
-      const Small<GP>* pr = cluster.map_shared_rank(&sm, r);
-      mx = max(mx, pr->maxpos);
-      fr = min(fr, pr->first_free);
-      er |= pr->err;
-    }
-    sm.g_t = mx + 1;
-    sm.g_free = fr;
-    sm.g_err = er;
-  }
-  __syncthreads();
-
-  // ----------------------------------------------- scores of own slots
-  const bool full_row = (sm.g_free == INT_MAX);
-  if (EVICT) {
-    unsigned long long k1 = kNoKey, k2 = kNoKey;
-    if (full_row && !sm.g_err) {
-      float w[G];
-#pragma unroll
-      for (int i = 0; i < G; ++i) w[i] = sm.cf[rank][i] / sm.Lg[i] * (1.0f / G);
-      const int lim = sm.g_t - p.window;
-      for (int j = tid; j < nvalid; j += kThreads) {
-        const int gj = slot0 + j;
-        if (gj < p.sink || pos_s[j] >= lim) continue;
-        float sc = 0.f;
-#pragma unroll
-        for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
-        top2_insert(k1, k2, (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) |
-                                static_cast<unsigned int>(gj));
-      }
-    }
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) {
-      const unsigned long long o1 = __shfl_xor_sync(0xffffffffu, k1, m);
-      const unsigned long long o2 = __shfl_xor_sync(0xffffffffu, k2, m);
-      top2_merge(k1, k2, o1, o2);
-    }
-    if (lane == 0) {
-      sm.wk1[warp] = k1;
-      sm.wk2[warp] = k2;
-    }
-  }
-
-  // ------------------------------------------ output: this CTA's share
-  {
-    constexpr int E = G * D;
-    const int per = (E + S - 1) / S;
-    const int e0 = rank * per, e1 = min(E, e0 + per);
-    const uint16_t* vn = p.v_new + size_t(row) * D;
-    for (int e = e0 + tid; e < e1; e += kThreads) {
-      const int i = e / D, d = e - i * D;
-      float acc = exp2f(sm.s_new[i] - sm.Mg[i]) * __uint_as_float(uint32_t(vn[d]) << 16);
-      for (int r = 0; r < S; ++r) acc = fmaf(cluster.map_shared_rank(xo, r)[e], sm.cf[r][i], acc);
-      p.out[size_t(row) * E + e] = acc / sm.Lg[i];
-    }
-  }
-
-  if (EVICT) {
-    __syncthreads();
-    if (tid == 0) {
-      unsigned long long k1 = kNoKey, k2 = kNoKey;
-      for (int w = 0; w < kWarps; ++w) top2_merge(k1, k2, sm.wk1[w], sm.wk2[w]);
-      sm.key1 = k1;
-      sm.key2 = k2;
-    }
-    cluster.sync();  // keys published
-    if (tid == 0) {
-      unsigned long long g1 = kNoKey, g2 = kNoKey;
-      for (int r = 0; r < S; ++r) {
-        const Small<GP>* pr = cluster.map_shared_rank(&sm, r);
-        top2_merge(g1, g2, pr->key1, pr->key2);
-      }
-      int refine = 0;
-      if (g1 != kNoKey && g2 != kNoKey) {
-        const float s1 = __uint_as_float(uint32_t(g1 >> 32));
-        const float s2 = __uint_as_float(uint32_t(g2 >> 32));
-        refine = (s2 <= s1 * (1.0f + kTieRel)) ? 1 : 0;
-      }
-      sm.g_refine = refine;
-      sm.g_slot = (g1 == kNoKey) ? -1 : int(uint32_t(g1 & 0xffffffffull));
-      // the published key1/key2 stay untouched: peers may still be reading them
-      sm.g_key1 = g1;
-    }
-    __syncthreads();
-
-    if (sm.g_refine) {  // identical decision in every CTA of the cluster
-      // fp64 rescoring of the candidates within the tie band
-      const float s1 = __uint_as_float(uint32_t(sm.g_key1 >> 32));
-      const float thr = s1 * (1.0f + kTieRel);
-      float w[G];
-#pragma unroll
-      for (int i = 0; i < G; ++i) w[i] = sm.cf[rank][i] / sm.Lg[i] * (1.0f / G);
-      const int lim = sm.g_t - p.window;
-      double best = INFINITY;
-      int bslot = INT_MAX;
-      for (int j = tid; j < nvalid; j += kThreads) {
-        const int gj = slot0 + j;
-        if (gj < p.sink || pos_s[j] >= lim) continue;
-        float sc = 0.f;
-#pragma unroll
-        for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
-        if (sc > thr) continue;
-        const uint16_t* krow = p.kcache + (size_t(row) * N + gj) * D;
-        double tot = 0.0;
         for (int i = 0; i < G; ++i) {
-          double dot = 0.0;
-          for (int d = 0; d < D; ++d) dot = fma(bf16_to_f64(qrow[i * D + d]), bf16_to_f64(krow[d]), dot);
-          tot += exp2(dot * p.qscale2_64 - double(sm.Mg[i])) / double(sm.Lg[i]);
-        }
-        tot /= double(G);
-        if (tot < best || (tot == best && gj < bslot)) {
-          best = tot;
-          bslot = gj;
+          float4* dst = reinterpret_cast<float4*>(red + (warp * G + i) * D + vsub * 8);
+          dst[0] = make_float4(o[i][0].x, o[i][0].y, o[i][1].x, o[i][1].y);
+          dst[1] = make_float4(o[i][2].x, o[i][2].y, o[i][3].x, o[i][3].y);
         }
       }
+      named_barrier(kBarConsumers, kConsumers);
+      {
+        float* xo = xo_buf(b);
+        for (int e = tid; e < G * D; e += kConsumers) {
+          float acc = 0.f;
 #pragma unroll
-      for (int m = 16; m > 0; m >>= 1) {
-        const double ob = __shfl_xor_sync(0xffffffffu, best, m);
-        const int os = __shfl_xor_sync(0xffffffffu, bslot, m);
-        if (ob < best || (ob == best && os < bslot)) {
-          best = ob;
-          bslot = os;
+          for (int w = 0; w < kCW; ++w) acc += red[w * G * D + e];
+          xo[e] = acc;
+        }
+        Pub<GP>* pb = pub_buf(b);
+        if (tid < G) {
+          float mm = -INFINITY, ll = 0.f;
+#pragma unroll
+          for (int w = 0; w < kCW; ++w) {
+            mm = fmaxf(mm, loc.wmax[w][tid]);
+            ll += loc.wsum[w][tid];
+          }
+          pb->m[tid] = mm;
+          pb->l[tid] = ll;
+        }
+        if (tid == 32) {
+          int mx = -1, fr = INT_MAX;
+#pragma unroll
+          for (int w = 0; w < kCW; ++w) {
+            mx = max(mx, loc.wpmax[w]);
+            fr = min(fr, loc.wpfree[w]);
+          }
+          pb->maxpos = mx;
+          pb->first_free = fr;
+          pb->err = loc.err;
         }
       }
-      if (lane == 0) {
-        sm.wref[warp] = best;
-        sm.wref_slot[warp] = bslot;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        double b = INFINITY;
-        int bs = INT_MAX;
-        for (int w2 = 0; w2 < kWarps; ++w2)
-          if (sm.wref[w2] < b || (sm.wref[w2] == b && sm.wref_slot[w2] < bs)) {
-            b = sm.wref[w2];
-            bs = sm.wref_slot[w2];
-          }
-        sm.ref_score = b;
-        sm.ref_slot = bs;
-      }
-      cluster.sync();  // rescoring results published
-      if (tid == 0) {
-        double b = INFINITY;
-        int bs = INT_MAX;
-        for (int r = 0; r < S; ++r) {
-          const Small<GP>* pr = cluster.map_shared_rank(&sm, r);
-          if (pr->ref_score < b || (pr->ref_score == b && pr->ref_slot < bs)) {
-            b = pr->ref_score;
-            bs = pr->ref_slot;
-          }
-        }
-        if (bs != INT_MAX) sm.g_slot = bs;
-      }
-      __syncthreads();
-    }
+      named_barrier(kBarConsumers, kConsumers);
 
-    // ------------------------------------------------ in-place eviction
-    if (rank == 0) {
-      int e, ev;
-      if (sm.g_err) {
-        e = -1;
-        ev = -2;
-      } else if (!full_row) {
-        e = sm.g_free;
-        ev = -1;
-      } else if (sm.g_slot < 0) {
-        e = -1;
-        ev = -2;
-        if (tid == 0) atomicOr(p.status, LF_STATUS_NO_CANDIDATE);
-      } else {
-        e = sm.g_slot;
-        ev = e;
-      }
-      if (e >= 0) {
-        constexpr int V16 = D / 8;  // 16-byte vectors per row
-        if (tid < V16) {
-          reinterpret_cast<uint4*>(p.kcache + (size_t(row) * N + e) * D)[tid] =
-              reinterpret_cast<const uint4*>(p.k_new + size_t(row) * D)[tid];
-        } else if (tid < 2 * V16) {
-          reinterpret_cast<uint4*>(p.vcache + (size_t(row) * N + e) * D)[tid - V16] =
-              reinterpret_cast<const uint4*>(p.v_new + size_t(row) * D)[tid - V16];
-        } else if (tid == 2 * V16) {
-          p.pos[size_t(row) * N + e] = sm.g_t;
+      // ------------------------------------------- exchange 1: max / sum
+      if (tid == 0) signal_cluster(&loc.xa[b], S);
+      wait_cl(&loc.xa[b], bpar);
+      if (warp == 0) {
+        const bool has = lane < S;
+        const Pub<GP>* pr = cluster.map_shared_rank(pub_buf(b), has ? lane : 0);
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          const float m = has ? pr->m[i] : -INFINITY;
+          float M = m;
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+          M = fmaxf(M, loc.s_new[i]);
+          const float cf = has ? exp2f(m - M) : 0.f;  // 0 for an empty chunk (m = -inf)
+          float lv = has ? pr->l[i] * cf : 0.f;
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o2);
+          if (has) loc.cf[lane][i] = cf;
+          if (lane == 0) {
+            loc.Mg[i] = M;
+            loc.Lg[i] = lv + exp2f(loc.s_new[i] - M);
+          }
+        }
+        int mx = has ? pr->maxpos : -1;
+        int fr = has ? pr->first_free : INT_MAX;
+        int er = has ? pr->err : 0;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) {
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+          fr = min(fr, __shfl_xor_sync(0xffffffffu, fr, o2));
+          er |= __shfl_xor_sync(0xffffffffu, er, o2);
+        }
+        if (lane == 0) {
+          loc.g_t = mx + 1;
+          loc.g_free = fr;
+          loc.g_err = er;
         }
       }
-      if (tid == 0) p.evicted[row] = ev;
+      named_barrier(kBarConsumers, kConsumers);
+      const bool full_row = (loc.g_free == INT_MAX);
+
+      // ------------------------------------------------ scores of own slots
+      if (EVICT) {
+        unsigned long long k1 = kNoKey, k2 = kNoKey;
+        if (full_row && !loc.g_err) {
+          float w[G];
+#pragma unroll
+          for (int i = 0; i < G; ++i) w[i] = loc.cf[rank][i] / loc.Lg[i] * (1.0f / G);
+          const int lim = loc.g_t - p.window;
+          for (int j = tid; j < nvalid; j += kConsumers) {
+            const int gj = slot0 + j;
+            if (gj < p.sink || ps[j] >= lim) continue;
+            float sc = 0.f;
+#pragma unroll
+            for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
+            top2_insert(k1, k2, (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) |
+                                    static_cast<unsigned int>(gj));
+          }
+        }
+        top2_warp(k1, k2);
+        if (lane == 0) {
+          loc.wk1[warp] = k1;
+          loc.wk2[warp] = k2;
+        }
+      }
+
+      // ------------------------------------------ output: this CTA's share
+      {
+        constexpr int E = G * D;
+        const int per = (E + S - 1) / S;
+        const int e0 = rank * per, e1 = min(E, e0 + per);
+        const uint16_t* vn = vn_buf(b);
+        for (int e = e0 + tid; e < e1; e += kConsumers) {
+          const int i = e / D, d = e - i * D;
+          float acc = exp2f(loc.s_new[i] - loc.Mg[i]) * __uint_as_float(uint32_t(vn[d]) << 16);
+          for (int r = 0; r < S; ++r)
+            acc = fmaf(cluster.map_shared_rank(xo_buf(b), r)[e], loc.cf[r][i], acc);
+          p.out[size_t(row) * E + e] = acc / loc.Lg[i];
+        }
+      }
+
+      if (EVICT) {
+        named_barrier(kBarConsumers, kConsumers);
+        if (warp == 0) {
+          unsigned long long k1 = lane < kCW ? loc.wk1[lane] : kNoKey;
+          unsigned long long k2 = lane < kCW ? loc.wk2[lane] : kNoKey;
+          top2_warp(k1, k2);
+          if (lane == 0) {
+            Pub<GP>* pb = pub_buf(b);
+            pb->key1 = k1;
+            pb->key2 = k2;
+          }
+        }
+        // ---------------------------------------- exchange 2: candidate keys
+        if (tid == 0) signal_cluster(&loc.xb[b], S);
+        wait_cl(&loc.xb[b], bpar);
+        if (warp == 0) {
+          const bool has = lane < S;
+          const Pub<GP>* pr = cluster.map_shared_rank(pub_buf(b), has ? lane : 0);
+          unsigned long long g1 = has ? pr->key1 : kNoKey;
+          unsigned long long g2 = has ? pr->key2 : kNoKey;
+          top2_warp(g1, g2);
+          if (lane == 0) {
+            int refine = 0;
+            if (g1 != kNoKey && g2 != kNoKey) {
+              const float s1 = __uint_as_float(uint32_t(g1 >> 32));
+              const float s2 = __uint_as_float(uint32_t(g2 >> 32));
+              refine = (s2 <= s1 * (1.0f + kTieRel)) ? 1 : 0;
+            }
+            loc.g_refine = refine;
+            loc.g_slot = (g1 == kNoKey) ? -1 : int(uint32_t(g1 & 0xffffffffull));
+            loc.g_key1 = g1;
+          }
+        }
+        named_barrier(kBarConsumers, kConsumers);
+
+        if (loc.g_refine) {  // the same decision in every CTA of the cluster
+          // fp64 rescoring of the candidates inside the tie band
+          const float s1 = __uint_as_float(uint32_t(loc.g_key1 >> 32));
+          const float thr = s1 * (1.0f + kTieRel);
+          float w[G];
+#pragma unroll
+          for (int i = 0; i < G; ++i) w[i] = loc.cf[rank][i] / loc.Lg[i] * (1.0f / G);
+          const int lim = loc.g_t - p.window;
+          const uint16_t* qs = q_buf(b);
+          double best = INFINITY;
+          int bslot = INT_MAX;
+          for (int j = tid; j < nvalid; j += kConsumers) {
+            const int gj = slot0 + j;
+            if (gj < p.sink || ps[j] >= lim) continue;
+            float sc = 0.f;
+#pragma unroll
+            for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
+            if (sc > thr) continue;
+            const uint16_t* krow = p.kcache + (size_t(row) * N + gj) * D;
+            double tot = 0.0;
+            for (int i = 0; i < G; ++i) {
+              double dot = 0.0;
+              for (int d = 0; d < D; ++d) dot = fma(bf16_to_f64(qs[i * D + d]), bf16_to_f64(krow[d]), dot);
+              tot += exp2(dot * p.qscale2_64 - double(loc.Mg[i])) / double(loc.Lg[i]);
+            }
+            tot /= double(G);
+            if (tot < best || (tot == best && gj < bslot)) {
+              best = tot;
+              bslot = gj;
+            }
+          }
+#pragma unroll
+          for (int m = 16; m > 0; m >>= 1) {
+            const double ob = __shfl_xor_sync(0xffffffffu, best, m);
+            const int os = __shfl_xor_sync(0xffffffffu, bslot, m);
+            if (ob < best || (ob == best && os < bslot)) {
+              best = ob;
+              bslot = os;
+            }
+          }
+          if (lane == 0) {
+            loc.wref[warp] = best;
+            loc.wrefs[warp] = bslot;
+          }
+          named_barrier(kBarConsumers, kConsumers);
+          if (warp == 0) {
+            double bb = lane < kCW ? loc.wref[lane] : INFINITY;
+            int bs = lane < kCW ? loc.wrefs[lane] : INT_MAX;
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) {
+              const double ob = __shfl_xor_sync(0xffffffffu, bb, m);
+              const int os = __shfl_xor_sync(0xffffffffu, bs, m);
+              if (ob < bb || (ob == bb && os < bs)) {
+                bb = ob;
+                bs = os;
+              }
+            }
+            if (lane == 0) {
+              Pub<GP>* pb = pub_buf(b);
+              pb->ref_score = bb;
+              pb->ref_slot = bs;
+            }
+          }
+          // ------------------------------------ exchange 3: fp64 rescoring
+          const uint32_t xpar = (b ? xc_uses1 : xc_uses0) & 1u;
+          if (b) ++xc_uses1;
+          else ++xc_uses0;
+          if (tid == 0) signal_cluster(&loc.xc[b], S);
+          wait_cl(&loc.xc[b], xpar);
+          if (warp == 0) {
+            const bool has = lane < S;
+            const Pub<GP>* pr = cluster.map_shared_rank(pub_buf(b), has ? lane : 0);
+            double bb = has ? pr->ref_score : INFINITY;
+            int bs = has ? pr->ref_slot : INT_MAX;
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) {
+              const double ob = __shfl_xor_sync(0xffffffffu, bb, m);
+              const int os = __shfl_xor_sync(0xffffffffu, bs, m);
+              if (ob < bb || (ob == bb && os < bs)) {
+                bb = ob;
+                bs = os;
+              }
+            }
+            if (lane == 0 && bs != INT_MAX) loc.g_slot = bs;
+          }
+          named_barrier(kBarConsumers, kConsumers);
+        }
+
+        // -------------------------------------------- in-place eviction
+        if (rank == 0) {
+          int e, ev;
+          if (loc.g_err || loc.err) {
+            e = -1;
+            ev = -2;
+          } else if (!full_row) {
+            e = loc.g_free;
+            ev = -1;
+          } else if (loc.g_slot < 0) {
+            e = -1;
+            ev = -2;
+            if (tid == 0) atomicOr(p.status, LF_STATUS_NO_CANDIDATE);
+          } else {
+            e = loc.g_slot;
+            ev = e;
+          }
+          if (e >= 0 && e < N) {
+            constexpr int V16 = D / 8;  // 16-byte vectors per row
+            if (tid < V16) {
+              reinterpret_cast<uint4*>(p.kcache + (size_t(row) * N + e) * D)[tid] =
+                  reinterpret_cast<const uint4*>(kn_buf(b))[tid];
+            } else if (tid < 2 * V16) {
+              reinterpret_cast<uint4*>(p.vcache + (size_t(row) * N + e) * D)[tid - V16] =
+                  reinterpret_cast<const uint4*>(vn_buf(b))[tid - V16];
+            } else if (tid == 2 * V16) {
+              p.pos[size_t(row) * N + e] = loc.g_t;
+            }
+          }
+          if (tid == 0) p.evicted[row] = ev;
+        }
+      }
+      // this row's logits, positions and metadata are no longer needed
+      named_barrier(kBarConsumers, kConsumers);
+      if (tid == 0) mbar_arrive(&loc.row_free[b]);
     }
   }
 
+  __syncthreads();
   // after an error, do not leave with bulk copies still landing in shared memory
-  if (sm.err && warp == kConsumerWarps && lane == 0) {
-    int nseq = 0;
-    for (int phase = 0; phase < 2; ++phase)
-      for (int tile = 0; tile < ntiles; ++tile) {
-        bool any = false;
-        for (int k = 0; k < T; ++k) {
-          const int j = tile * T + k;
-          any |= (j < nvalid) && (pos_s[j] >= 0);
-        }
-        nseq += any ? 1 : 0;
-      }
-    for (int q = max(0, nseq - kStages); q < nseq; ++q)
-      mbar_wait_bounded(&sm.full[q % kStages], uint32_t(q / kStages) & 1u, kWaitLimitNs);
+  if (loc.err && tid == kConsumers) {
+    for (int q = max(0, seq - nst); q < seq; ++q)
+      mbar_wait_bounded(&loc.full[q % nst], uint32_t(q / nst) & 1u, kWaitLimitNs);
   }
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }
@@ -747,6 +982,18 @@ __global__ void prefill_kernel(const uint4* __restrict__ k, const uint4* __restr
 // host side
 // ======================================================================
 
+namespace {
+
+// How one call is laid out on the GPU: S CTAs per row (one cluster), the
+// slots each CTA owns, the ring depth, and how many persistent clusters run.
+struct Plan {
+  int budget;  // the budget the plan was made for (0 = none)
+  int S, chunk, nstages, nclusters;
+  size_t smem;
+};
+
+}  // namespace
+
 struct lf_ctx {
   int B, Hq, Hkv, D, G, max_budget;
   cudaStream_t stream;
@@ -756,32 +1003,18 @@ struct lf_ctx {
   int split_override;
   int* status;  // device status word
   int last_bits;
+  Plan plan[2];  // [evict]
   unsigned magic;
 };
 
 namespace {
 
 constexpr unsigned kMagic = 0x4c46444bu;
+constexpr int kRowOverheadSlots = 256;  // per-row cost of the exchange, in slot units
 
 bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
 bool valid_handle(lf_handle h) { return h != nullptr && h->magic == kMagic; }
-
-template <int D, int G>
-size_t smem_for(int chunk) {
-  return lf::Geometry<D, G>::smem_bytes(chunk);
-}
-
-size_t smem_bytes(int D, int G, int chunk) {
-#define LF_CASE(DD, GG) \
-  if (D == DD && G == GG) return smem_for<DD, GG>(chunk);
-  LF_CASE(64, 1) LF_CASE(64, 2) LF_CASE(64, 3) LF_CASE(64, 4)
-  LF_CASE(64, 5) LF_CASE(64, 6) LF_CASE(64, 7) LF_CASE(64, 8)
-  LF_CASE(128, 1) LF_CASE(128, 2) LF_CASE(128, 3) LF_CASE(128, 4)
-  LF_CASE(128, 5) LF_CASE(128, 6) LF_CASE(128, 7) LF_CASE(128, 8)
-#undef LF_CASE
-  return 0;
-}
 
 int tile_slots(int D) { return lf::kTileBytes / (2 * D); }
 
@@ -791,49 +1024,82 @@ int chunk_for(int budget, int split, int D) {
   return ((per + T - 1) / T) * T;
 }
 
-// Split of one row over a cluster: enough CTAs to fill the GPU several
-// times over, chunks of at least 256 slots, and shared memory in budget.
-int choose_split(const lf_ctx* c, int budget) {
-  if (c->split_override > 0) return c->split_override;
+template <int D, int G, bool EVICT>
+cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
+  using Geo = lf::Geometry<D, G>;
+  auto kern = lf::fused_decode_kernel<D, G, EVICT>;
+  static std::mutex mu;
+  static bool attrs_set = false;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attrs_set) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           c->smem_optin);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      attrs_set = true;
+    }
+  }
   const int rows = c->B * c->Hkv;
-  int S = 1;
-  while (S < 8 && rows * S < 4 * c->sm_count && chunk_for(budget, 2 * S, c->D) >= 256) S *= 2;
-  // long rows: keep each CTA's chunk modest so several CTAs fit per SM
-  while (S < 8 && chunk_for(budget, S, c->D) > 512) S *= 2;
-  while (S < lf::kMaxSplit &&
-         smem_bytes(c->D, c->G, chunk_for(budget, S, c->D)) > size_t(c->smem_optin))
-    S *= 2;
-  return S;
+  Plan best = {};
+  long long best_cost = -1;
+  const int cands[5] = {1, 2, 4, 8, 16};
+  for (int ci = 0; ci < 5; ++ci) {
+    const int S = cands[ci];
+    if (c->split_override > 0 && S != c->split_override) continue;
+    const int chunk = chunk_for(budget, S, D);
+    const size_t fixed = Geo::layout(chunk, 0).total;
+    if (fixed + size_t(lf::kMinStages) * lf::kTileBytes > size_t(c->smem_optin)) continue;
+    int nst = int((size_t(c->smem_optin) - fixed) / lf::kTileBytes);
+    if (nst > lf::kMaxStages) nst = lf::kMaxStages;
+    const size_t smem = Geo::layout(chunk, nst).total;
+    if (smem > size_t(c->smem_optin)) continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(S), unsigned(rows), 1);
+    cfg.blockDim = dim3(lf::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess || ncl < 1) {
+      cudaGetLastError();  // clear a refused size
+      continue;
+    }
+    if (ncl > rows) ncl = rows;
+    const long long iters = (rows + ncl - 1) / ncl;
+    const long long cost = iters * (chunk + kRowOverheadSlots);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.S = S;
+      best.chunk = chunk;
+      best.nstages = nst;
+      best.nclusters = ncl;
+      best.smem = smem;
+    }
+  }
+  if (best_cost < 0) return cudaErrorInvalidConfiguration;
+  best.budget = budget;
+  *out = best;
+  return cudaSuccess;
 }
 
 template <int D, int G, bool EVICT>
-cudaError_t launch_t(const lf::Params& p, int rows, int S, size_t smem, cudaStream_t st) {
+cudaError_t launch_t(const lf::Params& p, const Plan& pl, cudaStream_t st) {
   auto kern = lf::fused_decode_kernel<D, G, EVICT>;
-  static std::mutex mu;
-  static size_t smem_set = 0;
-  static bool nonportable = false;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (smem > smem_set) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int(smem));
-      if (e != cudaSuccess) return e;
-      smem_set = smem;
-    }
-    if (S > 8 && !nonportable) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-      nonportable = true;
-    }
-  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(S), unsigned(rows), 1);
+  cfg.gridDim = dim3(unsigned(pl.S), unsigned(pl.nclusters), 1);
   cfg.blockDim = dim3(lf::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(S);
+  attr[0].val.clusterDim.x = unsigned(pl.S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -841,17 +1107,43 @@ cudaError_t launch_t(const lf::Params& p, int rows, int S, size_t smem, cudaStre
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-template <bool EVICT>
-cudaError_t launch(int D, int G, const lf::Params& p, int rows, int S, size_t smem,
-                   cudaStream_t st) {
-#define LF_CASE(DD, GG) \
-  if (D == DD && G == GG) return launch_t<DD, GG, EVICT>(p, rows, S, smem, st);
-  LF_CASE(64, 1) LF_CASE(64, 2) LF_CASE(64, 3) LF_CASE(64, 4)
-  LF_CASE(64, 5) LF_CASE(64, 6) LF_CASE(64, 7) LF_CASE(64, 8)
-  LF_CASE(128, 1) LF_CASE(128, 2) LF_CASE(128, 3) LF_CASE(128, 4)
-  LF_CASE(128, 5) LF_CASE(128, 6) LF_CASE(128, 7) LF_CASE(128, 8)
-#undef LF_CASE
-  return cudaErrorInvalidValue;
+#define LF_DISPATCH(D_, G_, CALL)                                                  \
+  do {                                                                             \
+    switch ((D_) * 16 + (G_)) {                                                    \
+      case 64 * 16 + 1: { constexpr int DD = 64, GG = 1; CALL; } break;            \
+      case 64 * 16 + 2: { constexpr int DD = 64, GG = 2; CALL; } break;            \
+      case 64 * 16 + 3: { constexpr int DD = 64, GG = 3; CALL; } break;            \
+      case 64 * 16 + 4: { constexpr int DD = 64, GG = 4; CALL; } break;            \
+      case 64 * 16 + 5: { constexpr int DD = 64, GG = 5; CALL; } break;            \
+      case 64 * 16 + 6: { constexpr int DD = 64, GG = 6; CALL; } break;            \
+      case 64 * 16 + 7: { constexpr int DD = 64, GG = 7; CALL; } break;            \
+      case 64 * 16 + 8: { constexpr int DD = 64, GG = 8; CALL; } break;            \
+      case 128 * 16 + 1: { constexpr int DD = 128, GG = 1; CALL; } break;          \
+      case 128 * 16 + 2: { constexpr int DD = 128, GG = 2; CALL; } break;          \
+      case 128 * 16 + 3: { constexpr int DD = 128, GG = 3; CALL; } break;          \
+      case 128 * 16 + 4: { constexpr int DD = 128, GG = 4; CALL; } break;          \
+      case 128 * 16 + 5: { constexpr int DD = 128, GG = 5; CALL; } break;          \
+      case 128 * 16 + 6: { constexpr int DD = 128, GG = 6; CALL; } break;          \
+      case 128 * 16 + 7: { constexpr int DD = 128, GG = 7; CALL; } break;          \
+      case 128 * 16 + 8: { constexpr int DD = 128, GG = 8; CALL; } break;          \
+      default: break;                                                              \
+    }                                                                              \
+  } while (0)
+
+cudaError_t get_plan(lf_ctx* c, int budget, bool evict, Plan** out) {
+  Plan& pl = c->plan[evict ? 1 : 0];
+  if (pl.budget != budget) {
+    cudaError_t e = cudaErrorInvalidValue;
+    pl.budget = 0;
+    if (evict) LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, true>(c, budget, &pl)));
+    else LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, false>(c, budget, &pl)));
+    if (e != cudaSuccess) {
+      pl.budget = 0;
+      return e;
+    }
+  }
+  *out = &pl;
+  return cudaSuccess;
 }
 
 int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
@@ -867,10 +1159,8 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
   if (evict && (sink < 0 || window < 1 || budget <= sink + window)) return LF_EINVAL;
 
-  const int S = choose_split(h, budget);
-  const int chunk = chunk_for(budget, S, h->D);
-  const size_t smem = smem_bytes(h->D, h->G, chunk);
-  if (smem > size_t(h->smem_optin)) return LF_EINVAL;
+  Plan* pl = nullptr;
+  if (get_plan(h, budget, evict, &pl) != cudaSuccess) return LF_ECUDA;
 
   lf::Params p;
   p.q = q;
@@ -882,17 +1172,19 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   p.out = out;
   p.evicted = evicted;
   p.status = h->status;
+  p.rows = h->B * h->Hkv;
   p.budget = budget;
-  p.chunk = chunk;
+  p.chunk = pl->chunk;
   p.sink = evict ? sink : 0;
   p.window = evict ? window : 1;
-  p.pos_vec4 = (budget % 4 == 0 && aligned(pos, 16)) ? 1 : 0;
+  p.nstages = pl->nstages;
+  p.pos_bulk = (budget % 4 == 0 && aligned(pos, 16)) ? 1 : 0;
   p.qscale2_64 = 1.4426950408889634 / sqrt(double(h->D));
   p.qscale2 = float(p.qscale2_64);
 
-  const int rows = h->B * h->Hkv;
-  cudaError_t e = evict ? launch<true>(h->D, h->G, p, rows, S, smem, h->stream)
-                        : launch<false>(h->D, h->G, p, rows, S, smem, h->stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  if (evict) LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, true>(p, *pl, h->stream)));
+  else LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, false>(p, *pl, h->stream)));
   return e == cudaSuccess ? LF_OK : LF_ECUDA;
 }
 
@@ -966,13 +1258,17 @@ int lf_set_split(lf_handle h, int split) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (split < 0 || split > lf::kMaxSplit || (split & (split - 1)) != 0) return LF_EINVAL;
   h->split_override = split;
+  h->plan[0].budget = 0;
+  h->plan[1].budget = 0;
   return LF_OK;
 }
 
 int lf_get_split(lf_handle h, int budget) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
-  return choose_split(h, budget);
+  Plan* pl = nullptr;
+  if (get_plan(h, budget, true, &pl) != cudaSuccess) return LF_ECUDA;
+  return pl->S;
 }
 
 int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, int n, uint16_t* kcache,
