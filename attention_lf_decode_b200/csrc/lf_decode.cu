@@ -94,20 +94,14 @@ struct Params {
   double qscale2_64;
 };
 
-// Per-CTA values that the other CTAs of the cluster read through
-// distributed shared memory (one copy per row parity).
+// What the CTAs of a cluster send each other about one row (one copy per
+// row parity, in every CTA).  Each CTA writes its own entries [rank] into
+// every CTA's copy with st.async; the receiver's mbarrier counts the bytes.
 template <int GP>
-struct Pub {
-  float m[GP];   // chunk max logit per head (log2 domain)
-  float l[GP];   // chunk sum of 2^(s - m) per head
-  int maxpos;    // newest position in the chunk (-1: none)
-  int first_free;
-  int err;
-  int pad0;
-  unsigned long long key1, key2;  // two lowest candidate keys
-  double ref_score;               // fp64 rescoring result
-  int ref_slot;
-  int pad1;
+struct Rx {
+  uint32_t sc[kMaxSplit][2 * GP + 4];     // per sender: m[GP], l[GP], maxpos, first_free, err
+  unsigned long long key[kMaxSplit][2];   // per sender: two lowest candidate keys
+  unsigned long long ref[kMaxSplit][2];   // per sender: fp64 rescoring (score bits, slot)
 };
 
 // CTA-local barriers and scalars.
@@ -117,9 +111,9 @@ struct Local {
   uint64_t empty[kMaxStages];
   uint64_t row_full[2];  // row metadata (positions, q, k_new, v_new) landed
   uint64_t row_free[2];  // consumers are done with a metadata buffer
-  uint64_t xa[2];        // cluster exchange: max / sum / positions published
-  uint64_t xb[2];        // cluster exchange: candidate keys published
-  uint64_t xc[2];        // cluster exchange: fp64 rescoring published
+  uint64_t xa[2];        // cluster exchange 1 received: max / sum / positions / partial output
+  uint64_t xb[2];        // cluster exchange 2 received: candidate keys
+  uint64_t xc[2];        // cluster exchange 3 received: fp64 rescoring
   float s_new[GP];
   float Mg[GP], Lg[GP];
   float cf[kMaxSplit][GP];
@@ -153,7 +147,8 @@ struct Geometry {
   static constexpr int VU = TPW / SPV;             // V phase: slot passes unrolled together
   static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
   static constexpr size_t kMetaStride = align128(size_t(G) * D * 2 + 2 * D * 2);
-  static constexpr size_t kPubStride = align128(size_t(G) * D * 4 + sizeof(Pub<GP>));
+  // per parity: this CTA's slice of every CTA's partial output, then Rx
+  static constexpr size_t kPubStride = align128(size_t(G) * D * 4) + align128(sizeof(Rx<GP>));
   static_assert(GROUPS % kCW == 0 && T % kCW == 0 && TPW % SPV == 0, "tile split");
 
   struct Layout {
@@ -176,6 +171,13 @@ struct Geometry {
 };
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+// 2^x on the SFU (flushes results below 2^-126 to zero; such probabilities
+// change no output, and equal zero scores are settled by the fp64 rescoring)
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ double bf16_to_f64(uint16_t b) {
   return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16));
@@ -241,6 +243,11 @@ __device__ __forceinline__ uint32_t map_rank(const void* p, int rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
   return r;
 }
+__device__ __forceinline__ uint32_t map_rank_addr(uint32_t smem_address, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_address), "r"(rank));
+  return r;
+}
 __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
@@ -248,11 +255,13 @@ __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
 __device__ __forceinline__ void fence_cluster() {
   asm volatile("fence.acq_rel.cluster;" ::: "memory");
 }
+// Non-blocking poll: a waiter suspended inside try_wait is not woken
+// promptly by arrivals from other CTAs, so cluster-level waits poll.
 __device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
       : "r"(smem_addr(bar)), "r"(parity)
@@ -264,16 +273,31 @@ __device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t par
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 64; ++i)
       if (try_wait_cluster(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
-// Signal barrier `bar` (same shared-memory offset in every CTA) of all S CTAs.
-__device__ __forceinline__ void signal_cluster(uint64_t* bar, int S) {
-  fence_cluster();
-  for (int r = 0; r < S; ++r) arrive_remote(map_rank(bar, r));
+// Asynchronous stores into the shared memory of a CTA of the cluster (this
+// one included), completing `bytes` on that CTA's mbarrier.  No release
+// fence is involved: a waiter that sees the mbarrier phase complete sees the
+// data.  Addresses are shared::cluster addresses from map_rank().
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr),
+               "r"(v), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_b64(uint32_t addr, unsigned long long v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(addr),
+               "l"(v), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+      : "memory");
 }
 
 // One reduce-scatter step over the 8 lanes of a slot.  The lane keeps the
@@ -343,9 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
   auto q_buf = [&](int b) { return reinterpret_cast<uint16_t*>(meta0 + b * Geo::kMetaStride); };
   auto kn_buf = [&](int b) { return q_buf(b) + G * D; };
   auto vn_buf = [&](int b) { return q_buf(b) + G * D + D; };
-  auto xo_buf = [&](int b) { return reinterpret_cast<float*>(pub0 + b * Geo::kPubStride); };
-  auto pub_buf = [&](int b) {
-    return reinterpret_cast<Pub<GP>*>(pub0 + b * Geo::kPubStride + size_t(G) * D * 4);
+  // [S][E / S] partial outputs of every sender for this CTA's output slice
+  auto rxo_buf = [&](int b) { return reinterpret_cast<float*>(pub0 + b * Geo::kPubStride); };
+  auto rx_buf = [&](int b) {
+    return reinterpret_cast<Rx<GP>*>(pub0 + b * Geo::kPubStride + align128(size_t(G) * D * 4));
   };
 
   if (tid == 0) {
@@ -357,9 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
     for (int b = 0; b < 2; ++b) {
       mbar_init(&loc.row_full[b], 1);
       mbar_init(&loc.row_free[b], 1);
-      mbar_init(&loc.xa[b], S);
-      mbar_init(&loc.xb[b], S);
-      mbar_init(&loc.xc[b], S);
+      mbar_init(&loc.xa[b], 1);  // the receiver's own expect-tx arrival + bytes
+      mbar_init(&loc.xb[b], 1);
+      mbar_init(&loc.xc[b], 1);
     }
     loc.err = 0;
     fence_mbar_init();
@@ -601,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           float pv = 0.f;
           if (eh < G) {
             const float x = pl[j * GP + eh];
-            pv = (x == -INFINITY) ? 0.f : exp2f(x - my_m);
+            pv = (x == -INFINITY) ? 0.f : ex2_ftz(x - my_m);
             pl[j * GP + eh] = pv;
           }
           lsum += pv;
@@ -671,15 +696,31 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
         }
       }
       named_barrier(kBarConsumers, kConsumers);
+
+      // ------------------- exchange 1: send this chunk's results to every CTA
+      // (the partial output goes by slices: CTA r combines elements
+      // [r * E / S, (r + 1) * E / S) of the row's output)
+      constexpr int E = G * D;
+      const int per = E / S;  // E is a multiple of 16 and S a power of two <= 16
       {
-        float* xo = xo_buf(b);
-        for (int e = tid; e < G * D; e += kConsumers) {
-          float acc = 0.f;
+        const uint32_t rxo_l = smem_addr(rxo_buf(b));
+        const uint32_t sc_l = smem_addr(&rx_buf(b)->sc[rank][0]);
+        const uint32_t bar_l = smem_addr(&loc.xa[b]);
+        for (int e4 = tid; e4 < E / 4; e4 += kConsumers) {
+          const int e = e4 * 4;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) acc += red[w * G * D + e];
-          xo[e] = acc;
+          for (int w = 0; w < kCW; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(red + w * E + e);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+          }
+          const int dst = e / per;
+          st_async_v4(map_rank_addr(rxo_l + uint32_t(rank * per + (e - dst * per)) * 4u, dst), acc,
+                      map_rank_addr(bar_l, dst));
         }
-        Pub<GP>* pb = pub_buf(b);
         if (tid < G) {
           float mm = -INFINITY, ll = 0.f;
 #pragma unroll
@@ -687,8 +728,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
             mm = fmaxf(mm, loc.wmax[w][tid]);
             ll += loc.wsum[w][tid];
           }
-          pb->m[tid] = mm;
-          pb->l[tid] = ll;
+          for (int r = 0; r < S; ++r) {
+            const uint32_t br = map_rank_addr(bar_l, r);
+            st_async_b32(map_rank_addr(sc_l + uint32_t(tid) * 4u, r), __float_as_uint(mm), br);
+            st_async_b32(map_rank_addr(sc_l + uint32_t(GP + tid) * 4u, r), __float_as_uint(ll), br);
+          }
         }
         if (tid == 32) {
           int mx = -1, fr = INT_MAX;
@@ -697,28 +741,31 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
             mx = max(mx, loc.wpmax[w]);
             fr = min(fr, loc.wpfree[w]);
           }
-          pb->maxpos = mx;
-          pb->first_free = fr;
-          pb->err = loc.err;
+          const int er = *reinterpret_cast<volatile int*>(&loc.err);
+          for (int r = 0; r < S; ++r) {
+            const uint32_t br = map_rank_addr(bar_l, r);
+            st_async_b32(map_rank_addr(sc_l + uint32_t(2 * GP) * 4u, r), uint32_t(mx), br);
+            st_async_b32(map_rank_addr(sc_l + uint32_t(2 * GP + 1) * 4u, r), uint32_t(fr), br);
+            st_async_b32(map_rank_addr(sc_l + uint32_t(2 * GP + 2) * 4u, r), uint32_t(er), br);
+          }
         }
       }
-      named_barrier(kBarConsumers, kConsumers);
-
-      // ------------------------------------------- exchange 1: max / sum
-      if (tid == 0) signal_cluster(&loc.xa[b], S);
-      wait_cl(&loc.xa[b], bpar);
+      // ----------- receive: every CTA's maxima, sums, positions (warp 0 waits)
       if (warp == 0) {
+        if (lane == 0)
+          mbar_arrive_expect_tx(&loc.xa[b], uint32_t(S) * uint32_t((2 * G + 3) * 4 + per * 4));
+        wait_cl(&loc.xa[b], bpar);
         const bool has = lane < S;
-        const Pub<GP>* pr = cluster.map_shared_rank(pub_buf(b), has ? lane : 0);
+        const uint32_t* sc = rx_buf(b)->sc[has ? lane : 0];
 #pragma unroll
         for (int i = 0; i < G; ++i) {
-          const float m = has ? pr->m[i] : -INFINITY;
+          const float m = has ? __uint_as_float(sc[i]) : -INFINITY;
           float M = m;
 #pragma unroll
           for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
           M = fmaxf(M, loc.s_new[i]);
           const float cf = has ? exp2f(m - M) : 0.f;  // 0 for an empty chunk (m = -inf)
-          float lv = has ? pr->l[i] * cf : 0.f;
+          float lv = has ? __uint_as_float(sc[GP + i]) * cf : 0.f;
 #pragma unroll
           for (int o2 = 16; o2 > 0; o2 >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o2);
           if (has) loc.cf[lane][i] = cf;
@@ -727,9 +774,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
             loc.Lg[i] = lv + exp2f(loc.s_new[i] - M);
           }
         }
-        int mx = has ? pr->maxpos : -1;
-        int fr = has ? pr->first_free : INT_MAX;
-        int er = has ? pr->err : 0;
+        int mx = has ? int(sc[2 * GP]) : -1;
+        int fr = has ? int(sc[2 * GP + 1]) : INT_MAX;
+        int er = has ? int(sc[2 * GP + 2]) : 0;
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) {
           mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
@@ -768,43 +815,43 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           loc.wk1[warp] = k1;
           loc.wk2[warp] = k2;
         }
+        named_barrier(kBarConsumers, kConsumers);
+        // ---------------------------- exchange 2: send the keys to every CTA
+        if (warp == 0) {
+          k1 = lane < kCW ? loc.wk1[lane] : kNoKey;
+          k2 = lane < kCW ? loc.wk2[lane] : kNoKey;
+          top2_warp(k1, k2);
+          if (lane < S) {
+            const uint32_t ka = map_rank_addr(smem_addr(&rx_buf(b)->key[rank][0]), lane);
+            const uint32_t br = map_rank_addr(smem_addr(&loc.xb[b]), lane);
+            st_async_b64(ka, k1, br);
+            st_async_b64(ka + 8u, k2, br);
+          }
+        }
       }
 
-      // ------------------------------------------ output: this CTA's share
+      // ------------------------------------------ output: this CTA's slice
       {
-        constexpr int E = G * D;
-        const int per = (E + S - 1) / S;
-        const int e0 = rank * per, e1 = min(E, e0 + per);
+        const int e0 = rank * per;
         const uint16_t* vn = vn_buf(b);
-        for (int e = e0 + tid; e < e1; e += kConsumers) {
+        const float* rxo = rxo_buf(b);
+        for (int k = tid; k < per; k += kConsumers) {
+          const int e = e0 + k;
           const int i = e / D, d = e - i * D;
           float acc = exp2f(loc.s_new[i] - loc.Mg[i]) * __uint_as_float(uint32_t(vn[d]) << 16);
-          for (int r = 0; r < S; ++r)
-            acc = fmaf(cluster.map_shared_rank(xo_buf(b), r)[e], loc.cf[r][i], acc);
+          for (int r = 0; r < S; ++r) acc = fmaf(rxo[r * per + k], loc.cf[r][i], acc);
           p.out[size_t(row) * E + e] = acc / loc.Lg[i];
         }
       }
 
       if (EVICT) {
-        named_barrier(kBarConsumers, kConsumers);
+        // ----------------------------------- receive: every CTA's keys
         if (warp == 0) {
-          unsigned long long k1 = lane < kCW ? loc.wk1[lane] : kNoKey;
-          unsigned long long k2 = lane < kCW ? loc.wk2[lane] : kNoKey;
-          top2_warp(k1, k2);
-          if (lane == 0) {
-            Pub<GP>* pb = pub_buf(b);
-            pb->key1 = k1;
-            pb->key2 = k2;
-          }
-        }
-        // ---------------------------------------- exchange 2: candidate keys
-        if (tid == 0) signal_cluster(&loc.xb[b], S);
-        wait_cl(&loc.xb[b], bpar);
-        if (warp == 0) {
+          if (lane == 0) mbar_arrive_expect_tx(&loc.xb[b], uint32_t(S) * 16u);
+          wait_cl(&loc.xb[b], bpar);
           const bool has = lane < S;
-          const Pub<GP>* pr = cluster.map_shared_rank(pub_buf(b), has ? lane : 0);
-          unsigned long long g1 = has ? pr->key1 : kNoKey;
-          unsigned long long g2 = has ? pr->key2 : kNoKey;
+          unsigned long long g1 = has ? rx_buf(b)->key[lane][0] : kNoKey;
+          unsigned long long g2 = has ? rx_buf(b)->key[lane][1] : kNoKey;
           top2_warp(g1, g2);
           if (lane == 0) {
             int refine = 0;
@@ -865,6 +912,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
             loc.wrefs[warp] = bslot;
           }
           named_barrier(kBarConsumers, kConsumers);
+          // -------------------- exchange 3: fp64 rescoring results to every CTA
+          const uint32_t xpar = (b ? xc_uses1 : xc_uses0) & 1u;
+          if (b) ++xc_uses1;
+          else ++xc_uses0;
           if (warp == 0) {
             double bb = lane < kCW ? loc.wref[lane] : INFINITY;
             int bs = lane < kCW ? loc.wrefs[lane] : INT_MAX;
@@ -877,23 +928,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
                 bs = os;
               }
             }
-            if (lane == 0) {
-              Pub<GP>* pb = pub_buf(b);
-              pb->ref_score = bb;
-              pb->ref_slot = bs;
+            if (lane < S) {
+              const uint32_t ra = map_rank_addr(smem_addr(&rx_buf(b)->ref[rank][0]), lane);
+              const uint32_t br = map_rank_addr(smem_addr(&loc.xc[b]), lane);
+              st_async_b64(ra, static_cast<unsigned long long>(__double_as_longlong(bb)), br);
+              st_async_b64(ra + 8u, static_cast<unsigned long long>(uint32_t(bs)), br);
             }
-          }
-          // ------------------------------------ exchange 3: fp64 rescoring
-          const uint32_t xpar = (b ? xc_uses1 : xc_uses0) & 1u;
-          if (b) ++xc_uses1;
-          else ++xc_uses0;
-          if (tid == 0) signal_cluster(&loc.xc[b], S);
-          wait_cl(&loc.xc[b], xpar);
-          if (warp == 0) {
+            if (lane == 0) mbar_arrive_expect_tx(&loc.xc[b], uint32_t(S) * 16u);
+            wait_cl(&loc.xc[b], xpar);
             const bool has = lane < S;
-            const Pub<GP>* pr = cluster.map_shared_rank(pub_buf(b), has ? lane : 0);
-            double bb = has ? pr->ref_score : INFINITY;
-            int bs = has ? pr->ref_slot : INT_MAX;
+            bb = has ? __longlong_as_double(static_cast<long long>(rx_buf(b)->ref[lane][0])) : INFINITY;
+            bs = has ? int(uint32_t(rx_buf(b)->ref[lane][1])) : INT_MAX;
 #pragma unroll
             for (int m = 16; m > 0; m >>= 1) {
               const double ob = __shfl_xor_sync(0xffffffffu, bb, m);
