@@ -878,33 +878,45 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           const uint16_t* qs = q_buf(b);
           double best = INFINITY;
           int bslot = INT_MAX;
-          for (int j = tid; j < nvalid; j += kConsumers) {
-            const int gj = slot0 + j;
-            if (gj < p.sink || ps[j] >= lim) continue;
-            float sc = 0.f;
+          // candidates inside the band are found 32 at a time per warp; each is
+          // then rescored by the whole warp (lane l: dims [l*D/32, (l+1)*D/32))
+          constexpr int DL = D / 32;
+          for (int base = warp * 32; base < nvalid; base += kConsumers) {
+            const int j = base + lane;
+            bool in_band = false;
+            if (j < nvalid) {
+              const int gj = slot0 + j;
+              if (gj >= p.sink && ps[j] < lim) {
+                float sc = 0.f;
 #pragma unroll
-            for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
-            if (sc > thr) continue;
-            const uint16_t* krow = p.kcache + (size_t(row) * N + gj) * D;
-            double tot = 0.0;
-            for (int i = 0; i < G; ++i) {
-              double dot = 0.0;
-              for (int d = 0; d < D; ++d) dot = fma(bf16_to_f64(qs[i * D + d]), bf16_to_f64(krow[d]), dot);
-              tot += exp2(dot * p.qscale2_64 - double(loc.Mg[i])) / double(loc.Lg[i]);
+                for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
+                in_band = sc <= thr;
+              }
             }
-            tot /= double(G);
-            if (tot < best || (tot == best && gj < bslot)) {
-              best = tot;
-              bslot = gj;
-            }
-          }
+            unsigned mask = __ballot_sync(0xffffffffu, in_band);
+            while (mask) {
+              const int src = __ffs(mask) - 1;
+              mask &= mask - 1;
+              const int gj = slot0 + base + src;
+              const uint16_t* krow = p.kcache + (size_t(row) * N + gj) * D + lane * DL;
+              double kv[DL];
 #pragma unroll
-          for (int m = 16; m > 0; m >>= 1) {
-            const double ob = __shfl_xor_sync(0xffffffffu, best, m);
-            const int os = __shfl_xor_sync(0xffffffffu, bslot, m);
-            if (ob < best || (ob == best && os < bslot)) {
-              best = ob;
-              bslot = os;
+              for (int d = 0; d < DL; ++d) kv[d] = bf16_to_f64(krow[d]);
+              double tot = 0.0;
+#pragma unroll
+              for (int i = 0; i < G; ++i) {
+                double dot = 0.0;
+#pragma unroll
+                for (int d = 0; d < DL; ++d) dot = fma(bf16_to_f64(qs[i * D + lane * DL + d]), kv[d], dot);
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
+                tot += exp2(dot * p.qscale2_64 - double(loc.Mg[i])) / double(loc.Lg[i]);
+              }
+              tot /= double(G);
+              if (tot < best || (tot == best && gj < bslot)) {
+                best = tot;
+                bslot = gj;
+              }
             }
           }
           if (lane == 0) {
