@@ -60,12 +60,11 @@ namespace cg = cooperative_groups;
 
 namespace lf {
 
-constexpr int kTileBytes = 32768;
 constexpr int kCW = 8;                      // consumer warps
 constexpr int kConsumers = kCW * 32;
 constexpr int kThreads = kConsumers + 32;   // + 1 producer warp
-constexpr int kMaxStages = 8;
-constexpr int kMinStages = 3;
+constexpr int kMaxStages = 4;
+constexpr int kMinStages = 2;
 constexpr int kMaxSplit = 16;
 constexpr int kMaxG = 8;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
@@ -132,8 +131,11 @@ __host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~si
 
 template <int D, int G>
 struct Geometry {
-  static constexpr int T = kTileBytes / (2 * D);   // slots per tile: 64 | 128
   static constexpr int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
+  // bytes per ring stage: large tiles amortise the per-tile work; the
+  // 8-head variants keep twice the probabilities per slot, so they take half
+  static constexpr int kTile = GP >= 8 ? 32768 : 65536;
+  static constexpr int T = kTile / (2 * D);        // slots per tile
   static constexpr int CPL = D / 64;               // K phase: 16-byte chunks per lane
   static constexpr int DPL = CPL * 8;              // K phase: dims per lane
   static constexpr int GROUPS = T / 4;             // K phase: 4-slot groups per tile
@@ -157,7 +159,7 @@ struct Geometry {
   __host__ __device__ static Layout layout(int chunk, int nst) {
     Layout L;
     size_t o = 0;
-    L.ring = o; o = align128(o + size_t(nst) * kTileBytes);
+    L.ring = o; o = align128(o + size_t(nst) * kTile);
     L.pl = o;   o = align128(o + size_t(chunk) * GP * 4);
     L.pos = o;  o = align128(o + size_t(2) * chunk * 4);
     L.red = o;  o = align128(o + size_t(kCW) * G * D * 4);
@@ -436,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           const int ns = min(T, nvalid - tile * T);
           const uint32_t bytes = uint32_t(ns) * D * 2;
           mbar_arrive_expect_tx(&loc.full[s], bytes);
-          bulk_copy_g2s(ring + size_t(s) * kTileBytes, base + size_t(tile) * T * D, bytes,
+          bulk_copy_g2s(ring + size_t(s) * Geo::kTile, base + size_t(tile) * T * D, bytes,
                         &loc.full[s]);
         }
         __syncwarp();
@@ -539,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           tfull = tile_full<T>(ps, tile, nvalid, lane);
         }
         wait_cta(&loc.full[stg], sph);
-        const unsigned char* kt = ring + size_t(stg) * kTileBytes;
+        const unsigned char* kt = ring + size_t(stg) * Geo::kTile;
 #pragma unroll 1
         for (int gb = 0; gb < GPW; gb += KU) {
           float xs[KU];
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           tfull = tile_full<T>(ps, tile, nvalid, lane);
         }
         wait_cta(&loc.full[stg], sph);
-        const unsigned char* vt = ring + size_t(stg) * kTileBytes;
+        const unsigned char* vt = ring + size_t(stg) * Geo::kTile;
         // probabilities of this warp's slots, kept for the scores and paired for the FMAs
 #pragma unroll
         for (int idx = lane; idx < TPW * GP; idx += 32) {
@@ -1073,10 +1075,7 @@ bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(pt
 
 bool valid_handle(lf_handle h) { return h != nullptr && h->magic == kMagic; }
 
-int tile_slots(int D) { return lf::kTileBytes / (2 * D); }
-
-int chunk_for(int budget, int split, int D) {
-  const int T = tile_slots(D);
+int chunk_for(int budget, int split, int T) {
   const int per = (budget + split - 1) / split;
   return ((per + T - 1) / T) * T;
 }
@@ -1105,10 +1104,10 @@ cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
   for (int ci = 0; ci < 5; ++ci) {
     const int S = cands[ci];
     if (c->split_override > 0 && S != c->split_override) continue;
-    const int chunk = chunk_for(budget, S, D);
+    const int chunk = chunk_for(budget, S, Geo::T);
     const size_t fixed = Geo::layout(chunk, 0).total;
-    if (fixed + size_t(lf::kMinStages) * lf::kTileBytes > size_t(c->smem_optin)) continue;
-    int nst = int((size_t(c->smem_optin) - fixed) / lf::kTileBytes);
+    if (fixed + size_t(lf::kMinStages) * Geo::kTile > size_t(c->smem_optin)) continue;
+    int nst = int((size_t(c->smem_optin) - fixed) / Geo::kTile);
     if (nst > lf::kMaxStages) nst = lf::kMaxStages;
     const size_t smem = Geo::layout(chunk, nst).total;
     if (smem > size_t(c->smem_optin)) continue;
@@ -1140,7 +1139,7 @@ cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
       best.smem = smem;
     }
   }
-  if (best_cost < 0) return cudaErrorInvalidConfiguration;
+  if (best_cost < 0) return cudaErrorInvalidConfiguration;  // no split fits: budget too large
   best.budget = budget;
   *out = best;
   return cudaSuccess;
@@ -1217,7 +1216,11 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   if (evict && (sink < 0 || window < 1 || budget <= sink + window)) return LF_EINVAL;
 
   Plan* pl = nullptr;
-  if (get_plan(h, budget, evict, &pl) != cudaSuccess) return LF_ECUDA;
+  {
+    const cudaError_t pe = get_plan(h, budget, evict, &pl);
+    if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
+    if (pe != cudaSuccess) return LF_ECUDA;
+  }
 
   lf::Params p;
   p.q = q;
@@ -1324,7 +1327,9 @@ int lf_get_split(lf_handle h, int budget) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
   Plan* pl = nullptr;
-  if (get_plan(h, budget, true, &pl) != cudaSuccess) return LF_ECUDA;
+  const cudaError_t pe = get_plan(h, budget, true, &pl);
+  if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
+  if (pe != cudaSuccess) return LF_ECUDA;
   return pl->S;
 }
 

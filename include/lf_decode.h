@@ -114,6 +114,9 @@ LF_API int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, i
  * has a candidate).  Positions in pos must be distinct; the kernel flags
  * LF_STATUS_NO_CANDIDATE, writes evicted = -2 and leaves the row's cache
  * unchanged when a full row has no candidate.
+ * A budget too large for one thread-block cluster of at most 16 CTAs to
+ * hold the row's logits in shared memory (about 32K slots at G = 4,
+ * D = 128; less for larger G) is rejected with LF_EINVAL.
  * Near ties: scores are computed in fp32; when the two lowest candidate
  * scores of a row are within a relative 1e-4 of each other, the kernel
  * rescores those candidates in fp64 before choosing. */
