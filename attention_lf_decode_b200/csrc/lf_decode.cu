@@ -60,9 +60,7 @@ namespace cg = cooperative_groups;
 
 namespace lf {
 
-constexpr int kCW = 8;                      // consumer warps
-constexpr int kConsumers = kCW * 32;
-constexpr int kThreads = kConsumers + 32;   // + 1 producer warp
+constexpr int kMaxCW = 11;                  // most consumer warps of any variant
 constexpr int kMaxStages = 4;
 constexpr int kMinStages = 2;
 constexpr int kMaxSplit = 16;
@@ -116,12 +114,12 @@ struct Local {
   float s_new[GP];
   float Mg[GP], Lg[GP];
   float cf[kMaxSplit][GP];
-  float wmax[kCW][GP];
-  float wsum[kCW][GP];
-  int wpmax[kCW], wpfree[kCW];
-  unsigned long long wk1[kCW], wk2[kCW];
-  double wref[kCW];
-  int wrefs[kCW];
+  float wmax[kMaxCW][GP];
+  float wsum[kMaxCW][GP];
+  int wpmax[kMaxCW], wpfree[kMaxCW];
+  unsigned long long wk1[kMaxCW], wk2[kMaxCW];
+  double wref[kMaxCW];
+  int wrefs[kMaxCW];
   unsigned long long g_key1;
   int g_t, g_free, g_err, g_refine, g_slot;
   int err;
@@ -132,26 +130,33 @@ __host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~si
 template <int D, int G>
 struct Geometry {
   static constexpr int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
-  // bytes per ring stage: large tiles amortise the per-tile work; the
-  // 8-head variants keep twice the probabilities per slot, so they take half
-  static constexpr int kTile = GP >= 8 ? 32768 : 65536;
+  // Consumer warps.  One SM runs one CTA; with 12 warps a scheduler holds 3,
+  // which leaves 168 registers per thread: 11 consumers + the producer.  The
+  // 8-head variants need more registers per thread and keep 8 consumers.
+  static constexpr int CW = GP >= 8 ? 8 : 11;
+  static constexpr int kConsumers = CW * 32;
+  static constexpr int kThreads = kConsumers + 32;  // + 1 producer warp
+  // Bytes per ring stage: large tiles amortise the per-tile work.  A tile
+  // holds 16 slots per consumer warp (176 at D = 128) for the small groups,
+  // 32 KB for the 8-head variants (which keep twice the probabilities).
+  static constexpr int kTile = GP >= 8 ? 32768 : CW * 16 * 2 * 128;
   static constexpr int T = kTile / (2 * D);        // slots per tile
   static constexpr int CPL = D / 64;               // K phase: 16-byte chunks per lane
   static constexpr int DPL = CPL * 8;              // K phase: dims per lane
   static constexpr int GROUPS = T / 4;             // K phase: 4-slot groups per tile
-  static constexpr int GPW = GROUPS / kCW;         // K phase: groups per warp per tile
+  static constexpr int GPW = GROUPS / CW;          // K phase: groups per warp per tile
   // K phase: groups computed together (more in flight hides latency; the
   // 8-head variants hold twice the query registers, so they take fewer)
   static constexpr int KU = GP >= 8 ? 1 : (GPW < 4 ? GPW : 4);
   static constexpr int VL = D / 8;                 // V phase: lanes per slot (8 dims each)
   static constexpr int SPV = 32 / VL;              // V phase: slots per warp pass
-  static constexpr int TPW = T / kCW;              // V phase: slots per warp per tile
+  static constexpr int TPW = T / CW;               // V phase: slots per warp per tile
   static constexpr int VU = TPW / SPV;             // V phase: slot passes unrolled together
   static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
   static constexpr size_t kMetaStride = align128(size_t(G) * D * 2 + 2 * D * 2);
   // per parity: this CTA's slice of every CTA's partial output, then Rx
   static constexpr size_t kPubStride = align128(size_t(G) * D * 4) + align128(sizeof(Rx<GP>));
-  static_assert(GROUPS % kCW == 0 && T % kCW == 0 && TPW % SPV == 0, "tile split");
+  static_assert(GROUPS % CW == 0 && T % CW == 0 && TPW % SPV == 0 && CW <= kMaxCW, "tile split");
 
   struct Layout {
     size_t ring, pl, pos, red, pp, meta, pub, loc, total;
@@ -160,10 +165,11 @@ struct Geometry {
     Layout L;
     size_t o = 0;
     L.ring = o; o = align128(o + size_t(nst) * kTile);
-    L.pl = o;   o = align128(o + size_t(chunk) * GP * 4);
+    // logits of whole tiles: the last tile of a chunk may be partial
+    L.pl = o;   o = align128(o + size_t((chunk + T - 1) / T * T) * GP * 4);
     L.pos = o;  o = align128(o + size_t(2) * chunk * 4);
-    L.red = o;  o = align128(o + size_t(kCW) * G * D * 4);
-    L.pp = o;   o = align128(o + size_t(kCW) * TPW * GP * 8);
+    L.red = o;  o = align128(o + size_t(CW) * G * D * 4);
+    L.pp = o;   o = align128(o + size_t(CW) * TPW * GP * 8);
     L.meta = o; o = align128(o + 2 * kMetaStride);
     L.pub = o;  o = align128(o + 2 * kPubStride);
     L.loc = o;  o = align128(o + sizeof(Local<GP>));
@@ -318,8 +324,9 @@ __device__ __forceinline__ void rs_step(float (&a)[kMaxG]) {
 }
 
 template <int D, int G, bool EVICT>
-__global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params p) {
+__global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kernel(const Params p) {
   using Geo = Geometry<D, G>;
+  constexpr int CW = Geo::CW, kConsumers = Geo::kConsumers;
   constexpr int T = Geo::T, GP = Geo::GP, CPL = Geo::CPL, DPL = Geo::DPL;
   constexpr int GPW = Geo::GPW, KU = Geo::KU, VU = Geo::VU, VL = Geo::VL, SPV = Geo::SPV,
                 TPW = Geo::TPW;
@@ -342,8 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
   unsigned char* ring = smem + L.ring;
   float* pl = reinterpret_cast<float*>(smem + L.pl);     // [chunk][GP] logits, then p
   int* pos0 = reinterpret_cast<int*>(smem + L.pos);      // [2][chunk]
-  float* red = reinterpret_cast<float*>(smem + L.red);   // [kCW][G][D]
-  float2* pp = reinterpret_cast<float2*>(smem + L.pp);   // [kCW][TPW][GP] (p, p) pairs
+  float* red = reinterpret_cast<float*>(smem + L.red);   // [CW][G][D]
+  float2* pp = reinterpret_cast<float2*>(smem + L.pp);   // [CW][TPW][GP] (p, p) pairs
   unsigned char* meta0 = smem + L.meta;                  // [2] {q[G][D], k_new[D], v_new[D]}
   unsigned char* pub0 = smem + L.pub;                    // [2] {xo[G][D], Pub}
   Local<GP>& loc = *reinterpret_cast<Local<GP>*>(smem + L.loc);
@@ -378,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&loc.full[s], 1);
-      mbar_init(&loc.empty[s], kCW);
+      mbar_init(&loc.empty[s], CW);
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
   int seq = 0, stg = 0;
   uint32_t sph = 0;
 
-  if (warp == kCW) {
+  if (warp == CW) {
     // ================================================================ producer
     auto issue_meta = [&](int it) {
       const int row = cid + it * ncl;
@@ -530,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
       named_barrier(kBarConsumers, kConsumers);
       bool fastrow = true;  // every slot of the chunk filled: no per-slot masking
 #pragma unroll
-      for (int w = 0; w < kCW; ++w) fastrow &= (loc.wpfree[w] == INT_MAX);
+      for (int w = 0; w < CW; ++w) fastrow &= (loc.wpfree[w] == INT_MAX);
 
       // ---------------------------------------------------------- K phase
       float rmax = -INFINITY;
@@ -547,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           float xs[KU];
 #pragma unroll
           for (int gu = 0; gu < KU; ++gu) {
-            const int si = (warp + (gb + gu) * kCW) * 4 + sig;
+            const int si = (warp + (gb + gu) * CW) * 4 + sig;
             float2 acc[GP];
 #pragma unroll
             for (int k = 0; k < GP; ++k) acc[k] = make_float2(0.f, 0.f);
@@ -575,13 +582,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
             const int ns = min(T, nvalid - tile * T);
 #pragma unroll
             for (int gu = 0; gu < KU; ++gu) {
-              const int si = (warp + (gb + gu) * kCW) * 4 + sig;
+              const int si = (warp + (gb + gu) * CW) * 4 + sig;
               if (!((si < ns) && (ps[tile * T + si] >= 0))) xs[gu] = -INFINITY;
             }
           }
 #pragma unroll
           for (int gu = 0; gu < KU; ++gu) {
-            const int j = tile * T + (warp + (gb + gu) * kCW) * 4 + sig;
+            const int j = tile * T + (warp + (gb + gu) * CW) * 4 + sig;
             if (kwriter) pl[j * GP + my_head] = xs[gu];
             rmax = fmaxf(rmax, xs[gu]);
           }
@@ -600,10 +607,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
       named_barrier(kBarConsumers, kConsumers);
 
       float my_m = -INFINITY;
-      if (eh < G) {
+      if (G == GP || eh < G) {
 #pragma unroll
-        for (int w = 0; w < kCW; ++w) my_m = fmaxf(my_m, loc.wmax[w][eh]);
+        for (int w = 0; w < CW; ++w) my_m = fmaxf(my_m, loc.wmax[w][eh]);
       }
+      // 2^(-inf - m) = 0 on the SFU, so masked slots need no select; only a
+      // head with no filled slot in the chunk (m = -inf) needs a finite offset
+      if (my_m == -INFINITY) my_m = 0.f;
 
       // ---------------------------------------------------------- V phase
       float2 o[G][4];
@@ -626,9 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
         for (int idx = lane; idx < TPW * GP; idx += 32) {
           const int j = tile * T + warp * TPW + idx / GP;
           float pv = 0.f;
-          if (eh < G) {
-            const float x = pl[j * GP + eh];
-            pv = (x == -INFINITY) ? 0.f : ex2_ftz(x - my_m);
+          if (G == GP || eh < G) {
+            pv = ex2_ftz(pl[j * GP + eh] - my_m);
             pl[j * GP + eh] = pv;
           }
           lsum += pv;
@@ -712,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           const int e = e4 * 4;
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) {
+          for (int w = 0; w < CW; ++w) {
             const float4 v = *reinterpret_cast<const float4*>(red + w * E + e);
             acc.x += v.x;
             acc.y += v.y;
@@ -726,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
         if (tid < G) {
           float mm = -INFINITY, ll = 0.f;
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) {
+          for (int w = 0; w < CW; ++w) {
             mm = fmaxf(mm, loc.wmax[w][tid]);
             ll += loc.wsum[w][tid];
           }
@@ -739,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
         if (tid == 32) {
           int mx = -1, fr = INT_MAX;
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) {
+          for (int w = 0; w < CW; ++w) {
             mx = max(mx, loc.wpmax[w]);
             fr = min(fr, loc.wpfree[w]);
           }
@@ -757,30 +766,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
         if (lane == 0)
           mbar_arrive_expect_tx(&loc.xa[b], uint32_t(S) * uint32_t((2 * G + 3) * 4 + per * 4));
         wait_cl(&loc.xa[b], bpar);
-        const bool has = lane < S;
-        const uint32_t* sc = rx_buf(b)->sc[has ? lane : 0];
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-          const float m = has ? __uint_as_float(sc[i]) : -INFINITY;
+        // all heads at once: lane = (head i, sender r) with S lanes per head
+        const int HP = 32 / S;  // heads per pass (S is a power of two <= 16)
+        for (int i0 = 0; i0 < G; i0 += HP) {
+          const int i = i0 + lane / S, r = lane % S;
+          const bool ok = i < G;
+          const uint32_t* sc = rx_buf(b)->sc[r];
+          const float m = ok ? __uint_as_float(sc[i]) : -INFINITY;
           float M = m;
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
-          M = fmaxf(M, loc.s_new[i]);
-          const float cf = has ? exp2f(m - M) : 0.f;  // 0 for an empty chunk (m = -inf)
-          float lv = has ? __uint_as_float(sc[GP + i]) * cf : 0.f;
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o2);
-          if (has) loc.cf[lane][i] = cf;
-          if (lane == 0) {
-            loc.Mg[i] = M;
-            loc.Lg[i] = lv + exp2f(loc.s_new[i] - M);
+          for (int o2 = 1; o2 < S; o2 <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+          const float sn = ok ? loc.s_new[i] : 0.f;
+          M = fmaxf(M, sn);
+          const float cf = ok ? exp2f(m - M) : 0.f;  // 0 for an empty chunk (m = -inf)
+          float lv = ok ? __uint_as_float(sc[GP + i]) * cf : 0.f;
+          for (int o2 = 1; o2 < S; o2 <<= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o2);
+          if (ok) {
+            loc.cf[r][i] = cf;
+            if (r == 0) {
+              loc.Mg[i] = M;
+              loc.Lg[i] = lv + exp2f(sn - M);
+            }
           }
         }
+        const bool has = lane < S;
+        const uint32_t* sc = rx_buf(b)->sc[has ? lane : 0];
         int mx = has ? int(sc[2 * GP]) : -1;
         int fr = has ? int(sc[2 * GP + 1]) : INT_MAX;
         int er = has ? int(sc[2 * GP + 2]) : 0;
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) {
+        for (int o2 = 1; o2 < S; o2 <<= 1) {
           mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
           fr = min(fr, __shfl_xor_sync(0xffffffffu, fr, o2));
           er |= __shfl_xor_sync(0xffffffffu, er, o2);
@@ -820,8 +833,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
         named_barrier(kBarConsumers, kConsumers);
         // ---------------------------- exchange 2: send the keys to every CTA
         if (warp == 0) {
-          k1 = lane < kCW ? loc.wk1[lane] : kNoKey;
-          k2 = lane < kCW ? loc.wk2[lane] : kNoKey;
+          k1 = lane < CW ? loc.wk1[lane] : kNoKey;
+          k2 = lane < CW ? loc.wk2[lane] : kNoKey;
           top2_warp(k1, k2);
           if (lane < S) {
             const uint32_t ka = map_rank_addr(smem_addr(&rx_buf(b)->key[rank][0]), lane);
@@ -931,8 +944,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const Params 
           if (b) ++xc_uses1;
           else ++xc_uses0;
           if (warp == 0) {
-            double bb = lane < kCW ? loc.wref[lane] : INFINITY;
-            int bs = lane < kCW ? loc.wrefs[lane] : INT_MAX;
+            double bb = lane < CW ? loc.wref[lane] : INFINITY;
+            int bs = lane < CW ? loc.wrefs[lane] : INT_MAX;
 #pragma unroll
             for (int m = 16; m > 0; m >>= 1) {
               const double ob = __shfl_xor_sync(0xffffffffu, bb, m);
@@ -1075,9 +1088,10 @@ bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(pt
 
 bool valid_handle(lf_handle h) { return h != nullptr && h->magic == kMagic; }
 
-int chunk_for(int budget, int split, int T) {
+// Slots per CTA: an even split, rounded up to 4 slots (16-byte position rows).
+int chunk_for(int budget, int split) {
   const int per = (budget + split - 1) / split;
-  return ((per + T - 1) / T) * T;
+  return (per + 3) / 4 * 4;
 }
 
 template <int D, int G, bool EVICT>
@@ -1104,7 +1118,7 @@ cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
   for (int ci = 0; ci < 5; ++ci) {
     const int S = cands[ci];
     if (c->split_override > 0 && S != c->split_override) continue;
-    const int chunk = chunk_for(budget, S, Geo::T);
+    const int chunk = chunk_for(budget, S);
     const size_t fixed = Geo::layout(chunk, 0).total;
     if (fixed + size_t(lf::kMinStages) * Geo::kTile > size_t(c->smem_optin)) continue;
     int nst = int((size_t(c->smem_optin) - fixed) / Geo::kTile);
@@ -1113,7 +1127,7 @@ cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
     if (smem > size_t(c->smem_optin)) continue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(S), unsigned(rows), 1);
-    cfg.blockDim = dim3(lf::kThreads, 1, 1);
+    cfg.blockDim = dim3(Geo::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1150,7 +1164,7 @@ cudaError_t launch_t(const lf::Params& p, const Plan& pl, cudaStream_t st) {
   auto kern = lf::fused_decode_kernel<D, G, EVICT>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(pl.S), unsigned(pl.nclusters), 1);
-  cfg.blockDim = dim3(lf::kThreads, 1, 1);
+  cfg.blockDim = dim3(lf::Geometry<D, G>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
