@@ -23,11 +23,20 @@ What one decode step computes, per row (batch entry b, KV head g), following
   section "Ограничения Памяти при Моделировании Длинных Последовательностей":
   one token is evicted after every attention computation.
 
-The score is fixed by the benchmark spec, not the pages: the softmax
-probability of the current query averaged over the G query heads of the KV
-group (the pages' alpha * ||v||_1 form ranks slots identically when all
-||v||_1 are equal).  The first ``sink`` slots and the last ``window``
-positions are protected; ties go to the lowest slot index.
+Two scores are offered (argument ``score``):
+
+* ``"mean_prob"`` (the default, fixed by the benchmark spec rather than the
+  pages): the softmax probability of the current query averaged over the G
+  query heads of the KV group;
+* ``"alpha_l1v"``: the summary page's own form, §2B: the attention weight
+  alpha of the token times the L1 norm of its value vector, sum_l |(v_j)_l|.
+  The page states it for one attention head; for a KV group read by G query
+  heads, alpha is read as the head-averaged probability, so this score is
+  the ``"mean_prob"`` score times ||v_j||_1.  Both rank slots identically
+  when every ||v_j||_1 is the same.
+
+The first ``sink`` slots and the last ``window`` positions are protected;
+ties go to the lowest slot index.
 
 Readings of points the pages leave open:
 
@@ -61,16 +70,22 @@ class RowStep:
     t: int                   # position written for the new token
     p: np.ndarray            # [G, N] probabilities of cached slots (0 where empty)
     p_new: np.ndarray        # [G] probability of the new token
-    score: Optional[np.ndarray]      # [N] head-averaged probability (None: no eviction)
+    score: Optional[np.ndarray]      # [N] eviction score of every slot (None: no eviction)
     candidates: Optional[np.ndarray]  # [N] bool, slots allowed to be evicted
 
 
-def decode_row(K, V, pos, q, k_new, v_new, sink: int, window: int) -> RowStep:
+SCORES = ("mean_prob", "alpha_l1v")
+
+
+def decode_row(K, V, pos, q, k_new, v_new, sink: int, window: int,
+               score: str = "mean_prob") -> RowStep:
     """One row of the decode step; inputs are not modified.
 
     K, V: [N, D] float64.  pos: [N] integer, -1 = empty.  q: [G, D].
-    k_new, v_new: [D].
+    k_new, v_new: [D].  score: one of SCORES.
     """
+    if score not in SCORES:
+        raise ValueError(f"unknown score {score!r}")
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
     q = np.asarray(q, np.float64)
@@ -107,13 +122,18 @@ def decode_row(K, V, pos, q, k_new, v_new, sink: int, window: int) -> RowStep:
         return RowStep(out, -1, slot, t, p, p_new, None, None)
 
     # zero-history score: this step's probability, averaged over the group
-    score = p.mean(axis=0)
+    alpha = p.mean(axis=0)
+    if score == "alpha_l1v":
+        # the page's form: alpha times the L1 norm of the slot's value vector
+        sc = alpha * np.abs(V).sum(axis=1)
+    else:
+        sc = alpha
     j = np.arange(N)
     cand = (j >= sink) & (pos < t - window)
     if not cand.any():
         raise ValueError("no slot may be evicted (sink + window cover the cache)")
-    slot = int(np.argmin(np.where(cand, score, np.inf)))  # first minimum = lowest index
-    return RowStep(out, slot, slot, t, p, p_new, score, cand)
+    slot = int(np.argmin(np.where(cand, sc, np.inf)))  # first minimum = lowest index
+    return RowStep(out, slot, slot, t, p, p_new, sc, cand)
 
 
 @dataclass
@@ -126,9 +146,11 @@ class StepResult:
     rows: list            # RowStep per (b, g), row-major
 
 
-def decode_step(kcache, vcache, pos, q, k_new, v_new, sink: int, window: int) -> StepResult:
+def decode_step(kcache, vcache, pos, q, k_new, v_new, sink: int, window: int,
+                score: str = "mean_prob") -> StepResult:
     """The batched decode step: kcache/vcache [B,Hkv,N,D], pos [B,Hkv,N],
-    q [B,Hq,D], k_new/v_new [B,Hkv,D].  Returns new arrays; inputs untouched."""
+    q [B,Hq,D], k_new/v_new [B,Hkv,D].  Returns new arrays; inputs untouched.
+    score: one of SCORES (see decode_row)."""
     kcache = np.array(kcache, np.float64, copy=True)
     vcache = np.array(vcache, np.float64, copy=True)
     pos = np.array(pos, np.int64, copy=True)
@@ -145,7 +167,7 @@ def decode_step(kcache, vcache, pos, q, k_new, v_new, sink: int, window: int) ->
         for g in range(Hkv):
             r = decode_row(kcache[b, g], vcache[b, g], pos[b, g],
                            q[b, g * G:(g + 1) * G], k_new[b, g], v_new[b, g],
-                           sink, window)
+                           sink, window, score)
             out[b, g * G:(g + 1) * G] = r.out
             evicted[b, g] = r.evicted
             kcache[b, g, r.slot] = k_new[b, g]

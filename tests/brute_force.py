@@ -4,14 +4,16 @@ Written from the definitions, independently of ``oracle/``: explicit loops,
 ``math.exp``, no NumPy arithmetic.  It is one of the pins of the oracle.
 Definitions: attention of the current query over the filled slots and the
 new token; score of a slot = its probability averaged over the query heads of
-the group; candidates = slot index >= sink and position older than the last
-``window`` positions; lowest score wins, lowest index on ties; a free slot
-(position -1) is filled first and then nothing is evicted.
+the group (``score="alpha_l1v"``: that average times the sum of the absolute
+values of the slot's value vector, the summary page's §2B form);
+candidates = slot index >= sink and position older than the last ``window``
+positions; lowest score wins, lowest index on ties; a free slot (position
+-1) is filled first and then nothing is evicted.
 """
 import math
 
 
-def brute_row(K, V, pos, q, k_new, v_new, sink, window):
+def brute_row(K, V, pos, q, k_new, v_new, sink, window, score="mean_prob"):
     """K, V: lists of N lists of D floats; pos: list of N ints; q: G lists.
 
     Returns (out [G][D], evicted, slot, t)."""
@@ -75,6 +77,11 @@ def brute_row(K, V, pos, q, k_new, v_new, sink, window):
         for i in range(G):
             sc += probs[i][j]
         sc /= G
+        if score == "alpha_l1v":
+            l1 = 0.0
+            for d in range(D):
+                l1 += abs(V[j][d])
+            sc *= l1
         if best is None or sc < best_score:
             best, best_score = j, sc
     if best is None:

@@ -8,6 +8,11 @@
   through slots sink .. sink + window;
 * hand-derived cases (tests/golden/hand_cases.json);
 * invariants of a whole trajectory and permutation equivariance.
+
+The page-form score (alpha times ||v||_1) has its own pins: the brute force,
+a hand case where it and the head-averaged probability disagree, a one-head
+closed form in the log domain (exact dot products, no softmax), zero-norm
+values, and equal-norm values (where it must rank exactly like the default).
 """
 import json
 import math
@@ -125,8 +130,9 @@ def test_probabilities_sum_to_one():
 
 # ------------------------------------------------------- P3: brute force
 
-@pytest.mark.parametrize("seed", range(40))
-def test_matches_scalar_brute_force(seed):
+@pytest.mark.parametrize("seed,score", [(s, "mean_prob") for s in range(40)]
+                         + [(s, "alpha_l1v") for s in range(100, 130)])
+def test_matches_scalar_brute_force(seed, score):
     rng = np.random.default_rng(seed)
     Hkv = int(rng.integers(1, 3))
     G = int(rng.integers(1, 4))
@@ -139,11 +145,11 @@ def test_matches_scalar_brute_force(seed):
         N = sink + window + 2
         fill = N
     K, V, pos, q, kn, vn = random_state(rng, 1, G * Hkv, Hkv, D, N, fill)
-    res = oracle.decode_step(K, V, pos, q, kn, vn, sink, window)
+    res = oracle.decode_step(K, V, pos, q, kn, vn, sink, window, score=score)
     for g in range(Hkv):
         out, ev, slot, t = brute_row(K[0, g].tolist(), V[0, g].tolist(), pos[0, g].tolist(),
                                      q[0, g * G:(g + 1) * G].tolist(), kn[0, g].tolist(),
-                                     vn[0, g].tolist(), sink, window)
+                                     vn[0, g].tolist(), sink, window, score=score)
         assert res.evicted[0, g] == ev
         assert res.rows[g].slot == slot and res.rows[g].t == t
         np.testing.assert_allclose(res.out[0, g * G:(g + 1) * G], np.array(out),
@@ -219,7 +225,8 @@ def test_hand_cases():
         q = np.array(c["q"], float)[None]
         kn = np.array(c["k_new"], float)[None, None]
         vn = np.array(c["v_new"], float)[None, None]
-        res = oracle.decode_step(K, V, pos, q, kn, vn, c["sink"], c["window"])
+        res = oracle.decode_step(K, V, pos, q, kn, vn, c["sink"], c["window"],
+                                 score=c.get("score", "mean_prob"))
         exp = c["expected"]
         r = res.rows[0]
         assert (res.evicted[0, 0], r.slot, r.t) == (exp["evicted"], exp["slot"], exp["t"]), c["name"]
@@ -330,3 +337,74 @@ def test_prefill_rejects_over_budget():
         oracle.prefill(np.zeros((1, 1, 5, 4)), np.zeros((1, 1, 5, 4)), 5, 4)
     kc, vc, pos = oracle.prefill(np.ones((1, 1, 3, 4)), np.ones((1, 1, 3, 4)), 3, 6)
     assert pos.tolist() == [[[0, 1, 2, -1, -1, -1]]]
+
+
+# ------------------------------------- the page-form score alpha * ||v||_1
+
+@pytest.mark.parametrize("seed", range(12))
+def test_page_score_single_head_log_domain(seed):
+    """G = 1: p_j = e^(s_j - m) / l with the same m and l for every slot, so
+    the page score p_j * ||v_j||_1 is lowest where s_j + ln ||v_j||_1 is
+    lowest.  s_j is an exact rational dot product; only the log is rounded."""
+    rng = np.random.default_rng(2000 + seed)
+    N, D, sink, window = 40, 16, 4, 8
+    K, V, pos, q, kn, vn = random_state(rng, 1, 1, 1, D, N, N)
+    V[0, 0] *= np.exp2(rng.integers(-3, 4, size=(N, 1)))  # spread the norms (exact in bf16)
+    res = oracle.decode_step(K, V, pos, q, kn, vn, sink, window, score="alpha_l1v")
+    t = int(pos.max()) + 1
+    scale = 1.0 / math.sqrt(D)
+    keyed = []
+    for j in range(N):
+        if j < sink or pos[0, 0, j] >= t - window:
+            continue
+        l1 = sum(Fraction(abs(float(x))) for x in V[0, 0, j])
+        keyed.append((float(_exact_dot(q[0, 0], K[0, 0, j])) * scale + math.log(float(l1)), j))
+    keyed.sort()
+    assert keyed[1][0] - keyed[0][0] > 1e-9  # no near tie in these draws
+    assert res.evicted[0, 0] == keyed[0][1]
+
+
+def test_page_score_zero_norm_values_go_first():
+    """A candidate whose value vector is all zeros scores exactly 0: the
+    lowest-index such candidate is evicted, whatever its probability."""
+    rng = np.random.default_rng(77)
+    N, D, sink, window = 24, 8, 2, 4
+    K, V, pos, q, kn, vn = random_state(rng, 1, 3, 1, D, N, N, permute=False)
+    V[0, 0, [1, 9, 14]] = 0.0   # slot 1 is a sink and may not go
+    K[0, 0, 14] = -K[0, 0, 14]  # whatever the logits
+    res = oracle.decode_step(K, V, pos, q, kn, vn, sink, window, score="alpha_l1v")
+    assert res.evicted[0, 0] == 9
+    assert res.rows[0].score[9] == 0.0 and res.rows[0].score[14] == 0.0
+
+
+def test_page_score_equal_norms_rank_like_mean_prob():
+    """With every ||v_j||_1 equal (values are signed permutations of one
+    vector) the two scores differ by one common factor, so a whole
+    trajectory evicts the same slots under both."""
+    rng = np.random.default_rng(78)
+    N, D, sink, window, G = 32, 8, 4, 6, 4
+    base = _bf16(rng, (D,))
+
+    def signed_perm():
+        return base[rng.permutation(D)] * rng.choice([-1.0, 1.0], size=D)
+
+    K = _bf16(rng, (1, 1, N, D))
+    V = np.stack([signed_perm() for _ in range(N)])[None, None]
+    pos = np.arange(N)[None, None].astype(np.int64)
+    Ka, Va, pa = K, V, pos
+    for k in range(60):
+        q = _bf16(rng, (1, G, D))
+        kn = _bf16(rng, (1, 1, D))
+        vn = signed_perm()[None, None]
+        ra = oracle.decode_step(Ka, Va, pa, q, kn, vn, sink, window, score="alpha_l1v")
+        rb = oracle.decode_step(Ka, Va, pa, q, kn, vn, sink, window, score="mean_prob")
+        assert ra.evicted[0, 0] == rb.evicted[0, 0], k
+        np.testing.assert_array_equal(ra.out, rb.out)
+        Ka, Va, pa = ra.kcache, ra.vcache, ra.pos
+
+
+def test_unknown_score_is_rejected():
+    rng = np.random.default_rng(3)
+    K, V, pos, q, kn, vn = random_state(rng, 1, 2, 1, 4, 8, 8)
+    with pytest.raises(ValueError):
+        oracle.decode_step(K, V, pos, q, kn, vn, 1, 2, score="l2")

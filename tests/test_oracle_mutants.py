@@ -24,11 +24,17 @@ MUTANTS = {
     "new_token_not_in_max": ("m = np.maximum(s.max(axis=1), s_new)", "m = s.max(axis=1)"),
     "scale_1_over_d": ("scale = 1.0 / math.sqrt(D)", "scale = 1.0 / D"),
     "gqa_strided_heads": ("q[b, g * G:(g + 1) * G], k_new[b, g]", "q[b, g::Hkv], k_new[b, g]"),
-    "score_max_over_heads": ("score = p.mean(axis=0)", "score = p.max(axis=0)"),
-    "score_first_head_only": ("score = p.mean(axis=0)", "score = p[0]"),
+    "score_max_over_heads": ("alpha = p.mean(axis=0)", "alpha = p.max(axis=0)"),
+    "score_first_head_only": ("alpha = p.mean(axis=0)", "alpha = p[0]"),
+    "l1v_signed_sum": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha * V.sum(axis=1)"),
+    "l1v_l2_norm": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha * np.sqrt((V * V).sum(axis=1))"),
+    "l1v_key_norm": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha * np.abs(K).sum(axis=1)"),
+    "l1v_divides": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha / np.abs(V).sum(axis=1)"),
+    "l1v_dropped": ('if score == "alpha_l1v":', 'if score == "no such score":'),
+    "l1v_max_norm": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha * np.abs(V).max(axis=1)"),
     "ties_to_highest_slot": (
-        "slot = int(np.argmin(np.where(cand, score, np.inf)))",
-        "slot = int(N - 1 - np.argmin(np.where(cand, score, np.inf)[::-1]))"),
+        "slot = int(np.argmin(np.where(cand, sc, np.inf)))",
+        "slot = int(N - 1 - np.argmin(np.where(cand, sc, np.inf)[::-1]))"),
     "t_is_max_pos": ("t = int(pos[filled].max()) + 1", "t = int(pos[filled].max())"),
     "append_to_highest_free": ("slot = int(np.flatnonzero(~filled)[0])",
                                "slot = int(np.flatnonzero(~filled)[-1])"),
@@ -56,8 +62,13 @@ def _pin_calls():
              (pins.test_hand_cases, {}),
              (pins.test_trajectory_invariants, {}),
              (pins.test_uniform_keys_evict_in_a_cycle, dict(N=32, sink=4, window=6, G=1))]
-    calls += [(pins.test_matches_scalar_brute_force, dict(seed=s)) for s in range(40)]
+    calls += [(pins.test_matches_scalar_brute_force, dict(seed=s, score="mean_prob")) for s in range(40)]
     calls += [(pins.test_single_head_evicts_lowest_exact_dot, dict(seed=s)) for s in range(4)]
+    calls += [(pins.test_matches_scalar_brute_force, dict(seed=s, score="alpha_l1v"))
+              for s in range(100, 130)]
+    calls += [(pins.test_page_score_single_head_log_domain, dict(seed=s)) for s in range(2)]
+    calls += [(pins.test_page_score_zero_norm_values_go_first, {}),
+              (pins.test_page_score_equal_norms_rank_like_mean_prob, {})]
     return calls
 
 
