@@ -23,9 +23,12 @@ LF_EDEVICE = -4
 LF_EUNSUPPORTED = -5
 LF_STATUS_WAIT_TIMEOUT = 1
 LF_STATUS_NO_CANDIDATE = 2
+LF_SCORE_MEAN_PROB = 0
+LF_SCORE_ALPHA_L1V = 1
 
 EXPORTS = ("lf_init", "lf_set_stream", "lf_prefill_cache", "lf_decode_step",
-           "lf_decode_attention", "lf_set_split", "lf_get_split", "lf_get_status",
+           "lf_decode_attention", "lf_set_split", "lf_get_split", "lf_set_score",
+           "lf_get_score", "lf_get_status",
            "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version",
            "lf_decode_step_noalloc")
 
@@ -57,6 +60,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lf_decode_attention": ([P, VP, VP, VP, VP, VP, VP, I, VP], I),
         "lf_set_split": ([P, I], I),
         "lf_get_split": ([P, I], I),
+        "lf_set_score": ([P, I], I),
+        "lf_get_score": ([P], I),
         "lf_get_status": ([P], I),
         "lf_status_bits": ([P], I),
         "lf_destroy": ([P], I),
@@ -148,6 +153,15 @@ def lf_set_split(h: Handle, split: int) -> None:
 
 def lf_get_split(h: Handle, budget: int) -> int:
     return _check(load_library().lf_get_split(h.ptr, budget), "lf_get_split")
+
+
+def lf_set_score(h: Handle, score: int) -> None:
+    """LF_SCORE_MEAN_PROB (default) or LF_SCORE_ALPHA_L1V (the page's form)."""
+    _check(load_library().lf_set_score(h.ptr, score), "lf_set_score")
+
+
+def lf_get_score(h: Handle) -> int:
+    return _check(load_library().lf_get_score(h.ptr), "lf_get_score")
 
 
 def lf_prefill_cache(h: Handle, k, v, n: int, kcache, vcache, pos, budget: int) -> None:

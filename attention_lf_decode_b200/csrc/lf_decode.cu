@@ -69,6 +69,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 constexpr float kTieRel = 1e-4f;                   // near-tie band rescored in fp64
 constexpr unsigned long long kNoKey = ~0ull;
 constexpr int kBarConsumers = 1;                   // named barrier of the consumer warps
+constexpr int kAttendOnly = 0, kEvictMeanProb = 1, kEvictAlphaL1V = 2;  // kernel modes
 
 struct Params {
   const uint16_t* q;
@@ -126,6 +127,7 @@ struct Local {
 };
 
 __host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 
 template <int D, int G>
 struct Geometry {
@@ -323,9 +325,14 @@ __device__ __forceinline__ void rs_step(float (&a)[kMaxG]) {
   }
 }
 
-template <int D, int G, bool EVICT>
+// MODE: kAttendOnly (attention, nothing scored or written), kEvictMeanProb
+// (evict the lowest head-averaged probability) or kEvictAlphaL1V (evict the
+// lowest head-averaged probability times the L1 norm of the slot's value).
+template <int D, int G, int MODE>
 __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kernel(const Params p) {
   using Geo = Geometry<D, G>;
+  constexpr bool EVICT = MODE != kAttendOnly;
+  constexpr bool L1V = MODE == kEvictAlphaL1V;
   constexpr int CW = Geo::CW, kConsumers = Geo::kConsumers;
   constexpr int T = Geo::T, GP = Geo::GP, CPL = Geo::CPL, DPL = Geo::DPL;
   constexpr int GPW = Geo::GPW, KU = Geo::KU, VU = Geo::VU, VL = Geo::VL, SPV = Geo::SPV,
@@ -471,6 +478,12 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
     const int my_head = perm;   // head whose logit this lane holds after the reduction
     const bool kwriter = ((sub & Geo::BFLY) == 0) && (my_head < G);
     const int vsub = lane % VL, vslot = lane / VL;
+    // Page-form score only: in V pass u this lane takes the warp's slot pair
+    // u ^ vperm instead of u, so that the per-slot L1 norms of a tile
+    // reduce-scatter over the slot's VL lanes without selects; afterwards
+    // the lane holds the norm of pass vperm's slot.
+    static_assert(VU <= VL && (VU & (VU - 1)) == 0, "norm reduce-scatter");
+    const int vperm = L1V ? (vsub >> (ilog2(VL) - ilog2(VU))) & (VU - 1) : 0;
     const int eh = lane % GP;   // head of this lane in the probability pass
     uint32_t xc_uses0 = 0, xc_uses1 = 0;
 
@@ -645,9 +658,10 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
         }
         __syncwarp();
         const int ns = tfull ? T : min(T, nvalid - tile * T);
+        float pn[kMaxG];  // page-form score: partial L1 norms, by pass
 #pragma unroll VU
         for (int u = 0; u < TPW / SPV; ++u) {
-          const int ls = u * SPV + vslot;
+          const int ls = (u ^ vperm) * SPV + vslot;
           const int si = warp * TPW + ls;
           const uint4 w = *reinterpret_cast<const uint4*>(vt + si * (2 * D) + vsub * 16);
           float2 v[4] = {make_float2(bf16lo(w.x), bf16hi(w.x)), make_float2(bf16lo(w.y), bf16hi(w.y)),
@@ -675,6 +689,30 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
           for (int i = 0; i < G; ++i)
 #pragma unroll
             for (int m = 0; m < 4; ++m) o[i][m] = __ffma2_rn(pi[i], v[m], o[i][m]);
+          if constexpr (L1V) {
+            float a = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) a += fabsf(v[m].x) + fabsf(v[m].y);
+            pn[u] = a;
+          }
+        }
+        if constexpr (L1V) {
+          // the page's score: fold ||v_j||_1 (from the tile already in shared
+          // memory) into the slot's stored probabilities
+          if constexpr (VL == 16) {
+            rs_step<VU, 8>(pn);
+            rs_step<(VU > 1 ? VU / 2 : 1), 4>(pn);
+            rs_step<(VU > 2 ? VU / 4 : 1), 2>(pn);
+            rs_step<(VU > 4 ? VU / 8 : 1), 1>(pn);
+          } else {
+            static_assert(VL == 8, "lanes per slot");
+            rs_step<VU, 4>(pn);
+            rs_step<(VU > 1 ? VU / 2 : 1), 2>(pn);
+            rs_step<(VU > 2 ? VU / 4 : 1), 1>(pn);
+          }
+          constexpr int DUP = VL / VU;  // lanes left holding the same slot's norm
+          const int j = tile * T + warp * TPW + vperm * SPV + vslot;
+          for (int i = vsub & (DUP - 1); i < G; i += DUP) pl[j * GP + i] *= pn[0];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&loc.empty[stg]);
@@ -928,6 +966,15 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
                 tot += exp2(dot * p.qscale2_64 - double(loc.Mg[i])) / double(loc.Lg[i]);
               }
               tot /= double(G);
+              if constexpr (L1V) {
+                const uint16_t* vrow = p.vcache + (size_t(row) * N + gj) * D + lane * DL;
+                double l1 = 0.0;
+#pragma unroll
+                for (int d = 0; d < DL; ++d) l1 += fabs(bf16_to_f64(vrow[d]));
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+                tot *= l1;
+              }
               if (tot < best || (tot == best && gj < bslot)) {
                 best = tot;
                 bslot = gj;
@@ -1075,7 +1122,8 @@ struct lf_ctx {
   int split_override;
   int* status;  // device status word
   int last_bits;
-  Plan plan[2];  // [evict]
+  int score_mode;  // LF_SCORE_* used by lf_decode_step
+  Plan plan[3];    // [kernel mode]
   unsigned magic;
 };
 
@@ -1094,10 +1142,10 @@ int chunk_for(int budget, int split) {
   return (per + 3) / 4 * 4;
 }
 
-template <int D, int G, bool EVICT>
+template <int D, int G, int MODE>
 cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
   using Geo = lf::Geometry<D, G>;
-  auto kern = lf::fused_decode_kernel<D, G, EVICT>;
+  auto kern = lf::fused_decode_kernel<D, G, MODE>;
   static std::mutex mu;
   static bool attrs_set = false;
   {
@@ -1159,9 +1207,9 @@ cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
   return cudaSuccess;
 }
 
-template <int D, int G, bool EVICT>
+template <int D, int G, int MODE>
 cudaError_t launch_t(const lf::Params& p, const Plan& pl, cudaStream_t st) {
-  auto kern = lf::fused_decode_kernel<D, G, EVICT>;
+  auto kern = lf::fused_decode_kernel<D, G, MODE>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(pl.S), unsigned(pl.nclusters), 1);
   cfg.blockDim = dim3(lf::Geometry<D, G>::kThreads, 1, 1);
@@ -1200,13 +1248,28 @@ cudaError_t launch_t(const lf::Params& p, const Plan& pl, cudaStream_t st) {
     }                                                                              \
   } while (0)
 
-cudaError_t get_plan(lf_ctx* c, int budget, bool evict, Plan** out) {
-  Plan& pl = c->plan[evict ? 1 : 0];
+// kernel mode of a call: attention only, or eviction by the handle's score
+int kernel_mode(const lf_ctx* c, bool evict) {
+  if (!evict) return lf::kAttendOnly;
+  return c->score_mode == LF_SCORE_ALPHA_L1V ? lf::kEvictAlphaL1V : lf::kEvictMeanProb;
+}
+
+cudaError_t get_plan(lf_ctx* c, int budget, int mode, Plan** out) {
+  Plan& pl = c->plan[mode];
   if (pl.budget != budget) {
     cudaError_t e = cudaErrorInvalidValue;
     pl.budget = 0;
-    if (evict) LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, true>(c, budget, &pl)));
-    else LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, false>(c, budget, &pl)));
+    switch (mode) {
+      case lf::kEvictMeanProb:
+        LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, lf::kEvictMeanProb>(c, budget, &pl)));
+        break;
+      case lf::kEvictAlphaL1V:
+        LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, lf::kEvictAlphaL1V>(c, budget, &pl)));
+        break;
+      default:
+        LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, lf::kAttendOnly>(c, budget, &pl)));
+        break;
+    }
     if (e != cudaSuccess) {
       pl.budget = 0;
       return e;
@@ -1229,9 +1292,10 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
   if (evict && (sink < 0 || window < 1 || budget <= sink + window)) return LF_EINVAL;
 
+  const int mode = kernel_mode(h, evict);
   Plan* pl = nullptr;
   {
-    const cudaError_t pe = get_plan(h, budget, evict, &pl);
+    const cudaError_t pe = get_plan(h, budget, mode, &pl);
     if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
     if (pe != cudaSuccess) return LF_ECUDA;
   }
@@ -1257,8 +1321,17 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   p.qscale2 = float(p.qscale2_64);
 
   cudaError_t e = cudaErrorInvalidValue;
-  if (evict) LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, true>(p, *pl, h->stream)));
-  else LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, false>(p, *pl, h->stream)));
+  switch (mode) {
+    case lf::kEvictMeanProb:
+      LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, lf::kEvictMeanProb>(p, *pl, h->stream)));
+      break;
+    case lf::kEvictAlphaL1V:
+      LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, lf::kEvictAlphaL1V>(p, *pl, h->stream)));
+      break;
+    default:
+      LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, lf::kAttendOnly>(p, *pl, h->stream)));
+      break;
+  }
   return e == cudaSuccess ? LF_OK : LF_ECUDA;
 }
 
@@ -1308,6 +1381,7 @@ int lf_init(lf_handle* out, int B, int Hq, int Hkv, int D, int max_budget, void*
   c->sm_count = prop.multiProcessorCount;
   c->smem_optin = int(prop.sharedMemPerBlockOptin);
   c->split_override = 0;
+  c->score_mode = LF_SCORE_MEAN_PROB;
   c->magic = kMagic;
   if (cudaMalloc(&c->status, sizeof(int)) != cudaSuccess) {
     free(c);
@@ -1332,16 +1406,27 @@ int lf_set_split(lf_handle h, int split) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (split < 0 || split > lf::kMaxSplit || (split & (split - 1)) != 0) return LF_EINVAL;
   h->split_override = split;
-  h->plan[0].budget = 0;
-  h->plan[1].budget = 0;
+  for (Plan& pl : h->plan) pl.budget = 0;
   return LF_OK;
+}
+
+int lf_set_score(lf_handle h, int score) {
+  if (!valid_handle(h)) return LF_ENOTINIT;
+  if (score != LF_SCORE_MEAN_PROB && score != LF_SCORE_ALPHA_L1V) return LF_EINVAL;
+  h->score_mode = score;
+  return LF_OK;
+}
+
+int lf_get_score(lf_handle h) {
+  if (!valid_handle(h)) return LF_ENOTINIT;
+  return h->score_mode;
 }
 
 int lf_get_split(lf_handle h, int budget) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
   Plan* pl = nullptr;
-  const cudaError_t pe = get_plan(h, budget, true, &pl);
+  const cudaError_t pe = get_plan(h, budget, kernel_mode(h, true), &pl);
   if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
   if (pe != cudaSuccess) return LF_ECUDA;
   return pl->S;

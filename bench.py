@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", default="throughput")
     ap.add_argument("--split", type=int, default=0, help="CTAs per row (0 = automatic)")
+    ap.add_argument("--score", default="mean_prob", choices=["mean_prob", "alpha_l1v"],
+                    help="eviction score: head-averaged probability (default) or the "
+                         "page's attention weight times the value L1 norm")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -164,7 +167,8 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle
 
-def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_steps: int):
+def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_steps: int,
+                score: str = "mean_prob"):
     """Time the CPU oracle, as it stands, on sampled batch entries; returns
     (full steps/s extrapolated from rows/s, sample description, steps run)."""
     import oracle
@@ -181,7 +185,7 @@ def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_s
         kn = synth.bf16_bits_to_f64(knb[batch_sel])
         vn = synth.bf16_bits_to_f64(vnb[batch_sel])
         t0 = time.perf_counter()
-        res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window)
+        res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window, score=score)
         t_total += time.perf_counter() - t0
         K, V, P = res.kcache, res.vcache, res.pos
         n += 1
@@ -240,6 +244,9 @@ def main():
     h = binding.lf_init(cfg.batch, cfg.hq, cfg.hkv, cfg.head_dim, cfg.budget, stream)
     if args.split:
         binding.lf_set_split(h, args.split)
+    score_code = {"mean_prob": binding.LF_SCORE_MEAN_PROB,
+                  "alpha_l1v": binding.LF_SCORE_ALPHA_L1V}[args.score]
+    binding.lf_set_score(h, score_code)
     split = binding.lf_get_split(h, cfg.budget)
     dev = "cuda"
     kcache = torch.empty((cfg.batch, cfg.hkv, cfg.budget, cfg.head_dim), dtype=torch.bfloat16, device=dev)
@@ -363,7 +370,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        rate, sample, _ = oracle_rate(cfg, gen, kpre, vpre, args.cpu_seconds, list(range(4)), 64)
+        rate, sample, _ = oracle_rate(cfg, gen, kpre, vpre, args.cpu_seconds, list(range(4)), 64,
+                                      score=args.score)
         cpu = {"value": rate, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
                "sample": sample}
 
@@ -384,6 +392,7 @@ def main():
             "window": cfg.window, "kv_dtype": "bf16", "accumulate": "f32",
             "parallelism": f"dp{world} (batch per rank, no collective)",
             "split_ctas_per_row": split,
+            "score": args.score,
             "l2": "inputs larger than L2: each step reads the 1 GiB K/V cache (L2 is 126 MB)",
             "tokens_per_s": value * cfg.batch,
             "us_per_step_per_layer": ms_per_step * 1e3,
@@ -394,7 +403,7 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
                      "bytes_per_launch": by["algorithmic"],
-                     "kernel": "lf::fused_decode_kernel<128,4,true>"},
+                     "kernel": f"lf::fused_decode_kernel<{cfg.head_dim},{cfg.group},{1 + score_code}>"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps,
@@ -437,7 +446,7 @@ def reference_arm(args, cfg, workload, world, rank):
         vn = synth.bf16_bits_to_f64(vnb[:1, :heads])
         t0 = time.perf_counter()
         res = oracle.decode_step(K[:, :heads], V[:, :heads], P[:, :heads], q, kn, vn,
-                                 cfg.sink, cfg.window)
+                                 cfg.sink, cfg.window, score=args.score)
         dt = time.perf_counter() - t0
         K[:, :heads], V[:, :heads], P[:, :heads] = res.kcache, res.vcache, res.pos
         if s >= args.warmup:
@@ -451,7 +460,8 @@ def reference_arm(args, cfg, workload, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": workload, "batch": cfg.batch, "budget": cfg.budget},
+        "config": {"workload": workload, "batch": cfg.batch, "budget": cfg.budget,
+                   "score": args.score},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

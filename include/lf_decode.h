@@ -70,6 +70,10 @@ extern "C" {
 #define LF_STATUS_WAIT_TIMEOUT 1  /* a bounded wait on a shared-memory barrier gave up */
 #define LF_STATUS_NO_CANDIDATE 2  /* full cache but no unprotected slot (corrupt pos table) */
 
+/* Eviction scores (lf_set_score) */
+#define LF_SCORE_MEAN_PROB 0  /* probability averaged over the group's query heads (default) */
+#define LF_SCORE_ALPHA_L1V 1  /* that average times the L1 norm of the slot's value vector */
+
 #if defined(__GNUC__)
 #define LF_API __attribute__((visibility("default")))
 #else
@@ -133,6 +137,23 @@ LF_API int lf_decode_attention(lf_handle h,
                         const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                         const uint16_t* kcache, const uint16_t* vcache, const int32_t* pos,
                         int budget, float* out);
+
+/* Eviction score used by later lf_decode_step calls on this handle.
+ *   LF_SCORE_MEAN_PROB (default): score_j as documented for lf_decode_step.
+ *   LF_SCORE_ALPHA_L1V: the LongFlow summary page's own form (§2B
+ *     "Derivación de la Métrica de Importancia"): the token's attention
+ *     weight times the L1 norm of its value vector, sum_l |v_j[l]|.  The
+ *     page states it for one head; for a KV group the weight is the
+ *     probability averaged over the group's query heads, so
+ *     score_j = mean_i p_ij * ||v_j||_1.  The norm is taken in the same pass
+ *     from the V tile already in shared memory; near ties are rescored in
+ *     fp64 with the norm recomputed in fp64.  Candidates, tie-break and
+ *     output are unchanged.
+ * Returns LF_EINVAL for any other value (the handle keeps its score). */
+LF_API int lf_set_score(lf_handle h, int score);
+
+/* The handle's eviction score (LF_SCORE_*), or a negative LF_E* code. */
+LF_API int lf_get_score(lf_handle h);
 
 /* Tuning: number of CTAs (a thread-block cluster) that split one row's
  * slots; 0 = automatic.  Must be 0 or a power of two <= 16. */

@@ -21,6 +21,8 @@ from attention_lf_decode_b200 import binding, synth
 
 OUT_ATOL = 2e-3
 TIE_REL = 1e-6
+# oracle score name -> the library's LF_SCORE_* code
+SCORE_CODES = {"mean_prob": binding.LF_SCORE_MEAN_PROB, "alpha_l1v": binding.LF_SCORE_ALPHA_L1V}
 
 
 @dataclass
@@ -38,7 +40,7 @@ class GpuCache:
     """Device-side cache of one config, driven through the C ABI."""
 
     def __init__(self, cfg: synth.DecodeConfig, prefill_k=None, prefill_v=None, n=None,
-                 split: int = 0, zero_init: bool = True):
+                 split: int = 0, zero_init: bool = True, score: str = "mean_prob"):
         import torch
         self.torch = torch
         self.cfg = cfg
@@ -48,6 +50,8 @@ class GpuCache:
         self.h = binding.lf_init(c.batch, c.hq, c.hkv, c.head_dim, c.budget)
         if split:
             binding.lf_set_split(self.h, split)
+        self.score = score
+        binding.lf_set_score(self.h, SCORE_CODES[score])
         self.kcache = alloc((c.batch, c.hkv, c.budget, c.head_dim), dtype=torch.bfloat16, device=dev)
         self.vcache = alloc((c.batch, c.hkv, c.budget, c.head_dim), dtype=torch.bfloat16, device=dev)
         self.pos = torch.full((c.batch, c.hkv, c.budget), -7, dtype=torch.int32, device=dev)
@@ -151,14 +155,14 @@ def check_step(res: "oracle.StepResult", pre_pos, gpu, stats: Stats, kbits_pre, 
 
 
 def teacher_forced(cfg: synth.DecodeConfig, steps: int, batch_idx=None, split: int = 0,
-                   gen: Optional[synth.SynthDecode] = None) -> Stats:
+                   gen: Optional[synth.SynthDecode] = None, score: str = "mean_prob") -> Stats:
     """Run `steps` decode steps on the GPU over the whole batch; after every
     step compare the rows of `batch_idx` with the oracle run from the same
     pre-step state.  Near-tie choices are accepted and the oracle follows the
     GPU's choice (the states stay identical)."""
     gen = gen or synth.SynthDecode(cfg)
     kpre, vpre = gen.prefill()
-    g = GpuCache(cfg, kpre, vpre, split=split)
+    g = GpuCache(cfg, kpre, vpre, split=split, score=score)
     bsel = list(range(cfg.batch)) if batch_idx is None else list(batch_idx)
     kb, vb = (synth.prefill_layout(kpre[bsel], vpre[bsel], cfg.budget)[:2])
     pos = synth.prefill_layout(kpre[bsel], vpre[bsel], cfg.budget)[2]
@@ -170,7 +174,8 @@ def teacher_forced(cfg: synth.DecodeConfig, steps: int, batch_idx=None, split: i
         K, V, P = oracle_state(kb, vb, pos)
         res = oracle.decode_step(K, V, P, synth.bf16_bits_to_f64(qb[bsel]),
                                  synth.bf16_bits_to_f64(knb[bsel]),
-                                 synth.bf16_bits_to_f64(vnb[bsel]), cfg.sink, cfg.window)
+                                 synth.bf16_bits_to_f64(vnb[bsel]), cfg.sink, cfg.window,
+                                 score=score)
         gpu = g.host_rows(None if batch_idx is None else bsel)
         kb, vb, pos = check_step(res, pos, gpu, stats, kb, vb, knb[bsel], vnb[bsel],
                                  where=f"{cfg.name} step {s}")
