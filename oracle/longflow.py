@@ -50,6 +50,9 @@ Readings of points the pages leave open:
 * A slot with pos < 0 is empty.  If any slot is empty the new token goes to
   the lowest empty slot and nothing is evicted (evicted = -1).
 * Query head h reads KV head h // G.
+* Ragged batches: a sequence may have a budget n_b below the allocated
+  slots N (``seq_budget``).  Its cache is then slots 0 .. n_b - 1 alone:
+  the slots beyond are neither read (not even for t) nor written.
 """
 from __future__ import annotations
 
@@ -147,10 +150,11 @@ class StepResult:
 
 
 def decode_step(kcache, vcache, pos, q, k_new, v_new, sink: int, window: int,
-                score: str = "mean_prob") -> StepResult:
+                score: str = "mean_prob", seq_budget=None) -> StepResult:
     """The batched decode step: kcache/vcache [B,Hkv,N,D], pos [B,Hkv,N],
     q [B,Hq,D], k_new/v_new [B,Hkv,D].  Returns new arrays; inputs untouched.
-    score: one of SCORES (see decode_row)."""
+    score: one of SCORES (see decode_row).  seq_budget: None, or [B] budgets
+    1 <= n_b <= N; batch entry b then uses slots 0 .. n_b - 1 only."""
     kcache = np.array(kcache, np.float64, copy=True)
     vcache = np.array(vcache, np.float64, copy=True)
     pos = np.array(pos, np.int64, copy=True)
@@ -160,12 +164,14 @@ def decode_step(kcache, vcache, pos, q, k_new, v_new, sink: int, window: int,
     if Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
     G = Hq // Hkv
+    nb = _seq_budgets(seq_budget, B, N)
     out = np.zeros((B, Hq, D))
     evicted = np.zeros((B, Hkv), np.int64)
     rows = []
     for b in range(B):
+        n = nb[b]
         for g in range(Hkv):
-            r = decode_row(kcache[b, g], vcache[b, g], pos[b, g],
+            r = decode_row(kcache[b, g, :n], vcache[b, g, :n], pos[b, g, :n],
                            q[b, g * G:(g + 1) * G], k_new[b, g], v_new[b, g],
                            sink, window, score)
             out[b, g * G:(g + 1) * G] = r.out
@@ -177,22 +183,34 @@ def decode_step(kcache, vcache, pos, q, k_new, v_new, sink: int, window: int,
     return StepResult(out, evicted, kcache, vcache, pos, rows)
 
 
-def decode_attention(kcache, vcache, pos, q, k_new, v_new) -> np.ndarray:
+def _seq_budgets(seq_budget, B: int, N: int) -> list:
+    if seq_budget is None:
+        return [N] * B
+    nb = [int(x) for x in np.asarray(seq_budget).reshape(-1)]
+    if len(nb) != B or any(n < 1 or n > N for n in nb):
+        raise ValueError("seq_budget needs B entries in 1 .. N")
+    return nb
+
+
+def decode_attention(kcache, vcache, pos, q, k_new, v_new, seq_budget=None) -> np.ndarray:
     """Plain single-query decode attention over filled slots + the new token
-    (the no-eviction control); nothing is scored or written."""
+    (the no-eviction control); nothing is scored or written.  seq_budget as
+    in decode_step."""
     kcache = np.asarray(kcache, np.float64)
     vcache = np.asarray(vcache, np.float64)
     pos = np.asarray(pos)
     q = np.asarray(q, np.float64)
     B, Hkv, N, D = kcache.shape
     G = q.shape[1] // Hkv
+    nb = _seq_budgets(seq_budget, B, N)
     out = np.zeros(q.shape)
     scale = 1.0 / math.sqrt(D)
     for b in range(B):
+        n = nb[b]
         for g in range(Hkv):
-            f = pos[b, g] >= 0
-            Kf = np.concatenate([kcache[b, g][f], np.asarray(k_new[b, g], np.float64)[None]])
-            Vf = np.concatenate([vcache[b, g][f], np.asarray(v_new[b, g], np.float64)[None]])
+            f = pos[b, g, :n] >= 0
+            Kf = np.concatenate([kcache[b, g, :n][f], np.asarray(k_new[b, g], np.float64)[None]])
+            Vf = np.concatenate([vcache[b, g, :n][f], np.asarray(v_new[b, g], np.float64)[None]])
             qs = q[b, g * G:(g + 1) * G]
             s = (qs @ Kf.T) * scale
             s -= s.max(axis=1, keepdims=True)

@@ -408,3 +408,82 @@ def test_unknown_score_is_rejected():
     K, V, pos, q, kn, vn = random_state(rng, 1, 2, 1, 4, 8, 8)
     with pytest.raises(ValueError):
         oracle.decode_step(K, V, pos, q, kn, vn, 1, 2, score="l2")
+
+
+# ------------------------------------------ ragged batches (per-sequence budget)
+
+def _ragged_state(rng, B, Hq, Hkv, D, N, sink, window):
+    """Per batch entry b a budget n_b; slots 0..n_b-1 hold a cache that is
+    full or partly free; the slots beyond hold junk that must be ignored:
+    NaN values and positions far above the prefix's."""
+    K, V, pos, q, kn, vn = random_state(rng, B, Hq, Hkv, D, N, N)
+    nb = rng.integers(sink + window + 1, N + 1, size=B)
+    for b in range(B):
+        n = int(nb[b])
+        full = rng.random() < 0.7
+        fill = n if full else int(rng.integers(0, n))
+        for g in range(Hkv):
+            pos[b, g, :n] = -1
+            slots = rng.permutation(n)[:fill]
+            pos[b, g, slots] = rng.permutation(fill) + int(rng.integers(0, 50))
+            pos[b, g, n:] = 10_000 + np.arange(N - n)
+            K[b, g, n:] = np.nan
+            V[b, g, n:] = np.nan
+    return K, V, pos, q, kn, vn, nb
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_ragged_matches_brute_force(seed):
+    rng = np.random.default_rng(3000 + seed)
+    B, Hkv, G = 3, int(rng.integers(1, 3)), int(rng.integers(1, 4))
+    D, N, sink, window = int(rng.choice([2, 4, 8])), int(rng.integers(8, 15)), 1, 2
+    score = "alpha_l1v" if seed % 2 else "mean_prob"
+    K, V, pos, q, kn, vn, nb = _ragged_state(rng, B, G * Hkv, Hkv, D, N, sink, window)
+    res = oracle.decode_step(K, V, pos, q, kn, vn, sink, window, score=score, seq_budget=nb)
+    for b in range(B):
+        n = int(nb[b])
+        for g in range(Hkv):
+            out, ev, slot, t = brute_row(K[b, g, :n].tolist(), V[b, g, :n].tolist(),
+                                         pos[b, g, :n].tolist(),
+                                         q[b, g * G:(g + 1) * G].tolist(), kn[b, g].tolist(),
+                                         vn[b, g].tolist(), sink, window, score=score)
+            assert res.evicted[b, g] == ev and res.rows[b * Hkv + g].t == t
+            np.testing.assert_allclose(res.out[b, g * G:(g + 1) * G], np.array(out),
+                                       rtol=0, atol=1e-12)
+            assert res.pos[b, g, slot] == t
+            # the junk beyond the budget is untouched (NaN stays NaN)
+            np.testing.assert_array_equal(res.pos[b, g, n:], pos[b, g, n:])
+            assert np.isnan(res.kcache[b, g, n:]).all() and np.isnan(res.vcache[b, g, n:]).all()
+
+
+def test_ragged_outputs_match_library_attention():
+    rng = np.random.default_rng(3100)
+    B, Hq, Hkv, D, N = 4, 8, 2, 16, 40
+    K, V, pos, q, kn, vn, nb = _ragged_state(rng, B, Hq, Hkv, D, N, 2, 4)
+    res = oracle.decode_step(K, V, pos, q, kn, vn, 2, 4, seq_budget=nb)
+    att = oracle.decode_attention(K, V, pos, q, kn, vn, seq_budget=nb)
+    for b in range(B):
+        n = int(nb[b])
+        ref = sdpa_reference(K[b:b + 1, :, :n], V[b:b + 1, :, :n], pos[b:b + 1, :, :n],
+                             q[b:b + 1], kn[b:b + 1], vn[b:b + 1])
+        np.testing.assert_allclose(res.out[b:b + 1], ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(att[b:b + 1], ref, rtol=0, atol=1e-12)
+    assert not np.isnan(res.out).any()
+
+
+def test_ragged_budget_equal_to_slots_is_the_plain_step():
+    rng = np.random.default_rng(3200)
+    K, V, pos, q, kn, vn = random_state(rng, 3, 6, 2, 8, 20, 20)
+    a = oracle.decode_step(K, V, pos, q, kn, vn, 2, 3)
+    b = oracle.decode_step(K, V, pos, q, kn, vn, 2, 3, seq_budget=[20, 20, 20])
+    np.testing.assert_array_equal(a.out, b.out)
+    np.testing.assert_array_equal(a.evicted, b.evicted)
+    np.testing.assert_array_equal(a.pos, b.pos)
+
+
+@pytest.mark.parametrize("nb", [[0, 5], [5, 21], [5]])
+def test_ragged_budget_validation(nb):
+    rng = np.random.default_rng(3300)
+    K, V, pos, q, kn, vn = random_state(rng, 2, 2, 1, 4, 20, 20)
+    with pytest.raises(ValueError):
+        oracle.decode_step(K, V, pos, q, kn, vn, 1, 2, seq_budget=nb)

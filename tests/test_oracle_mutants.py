@@ -32,6 +32,10 @@ MUTANTS = {
     "l1v_divides": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha / np.abs(V).sum(axis=1)"),
     "l1v_dropped": ('if score == "alpha_l1v":', 'if score == "no such score":'),
     "l1v_max_norm": ("sc = alpha * np.abs(V).sum(axis=1)", "sc = alpha * np.abs(V).max(axis=1)"),
+    "ragged_budget_ignored": ("        n = nb[b]\n        for g in range(Hkv):\n            r = decode_row(",
+                              "        n = N\n        for g in range(Hkv):\n            r = decode_row("),
+    "ragged_budget_minus_one": ("        n = nb[b]\n        for g in range(Hkv):\n            r = decode_row(",
+                                "        n = max(1, nb[b] - 1)\n        for g in range(Hkv):\n            r = decode_row("),
     "ties_to_highest_slot": (
         "slot = int(np.argmin(np.where(cand, sc, np.inf)))",
         "slot = int(N - 1 - np.argmin(np.where(cand, sc, np.inf)[::-1]))"),
@@ -67,6 +71,8 @@ def _pin_calls():
     calls += [(pins.test_matches_scalar_brute_force, dict(seed=s, score="alpha_l1v"))
               for s in range(100, 130)]
     calls += [(pins.test_page_score_single_head_log_domain, dict(seed=s)) for s in range(2)]
+    calls += [(pins.test_ragged_matches_brute_force, dict(seed=s)) for s in range(6)]
+    calls += [(pins.test_ragged_outputs_match_library_attention, {})]
     calls += [(pins.test_page_score_zero_norm_values_go_first, {}),
               (pins.test_page_score_equal_norms_rank_like_mean_prob, {})]
     return calls
