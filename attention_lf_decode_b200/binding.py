@@ -23,11 +23,12 @@ LF_EDEVICE = -4
 LF_EUNSUPPORTED = -5
 LF_STATUS_WAIT_TIMEOUT = 1
 LF_STATUS_NO_CANDIDATE = 2
+LF_STATUS_BAD_SEQ_BUDGET = 4
 LF_SCORE_MEAN_PROB = 0
 LF_SCORE_ALPHA_L1V = 1
 
 EXPORTS = ("lf_init", "lf_set_stream", "lf_prefill_cache", "lf_decode_step",
-           "lf_decode_attention", "lf_set_split", "lf_get_split", "lf_set_score",
+           "lf_decode_attention", "lf_decode_step_ragged", "lf_decode_attention_ragged", "lf_set_split", "lf_get_split", "lf_set_score",
            "lf_get_score", "lf_get_status",
            "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version",
            "lf_decode_step_noalloc")
@@ -58,6 +59,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lf_prefill_cache": ([P, VP, VP, I, VP, VP, VP, I], I),
         "lf_decode_step": ([P, VP, VP, VP, VP, VP, VP, I, I, I, VP, VP], I),
         "lf_decode_attention": ([P, VP, VP, VP, VP, VP, VP, I, VP], I),
+        "lf_decode_step_ragged": ([P, VP, VP, VP, VP, VP, VP, I, VP, I, I, VP, VP], I),
+        "lf_decode_attention_ragged": ([P, VP, VP, VP, VP, VP, VP, I, VP, VP], I),
         "lf_set_split": ([P, I], I),
         "lf_get_split": ([P, I], I),
         "lf_set_score": ([P, I], I),
@@ -199,6 +202,37 @@ def lf_decode_attention(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget:
         _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
         _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
         _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention")
+
+
+def lf_decode_step_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
+                          seq_budget, sink: int, window: int, out, evicted_idx) -> None:
+    """lf_decode_step with a per-sequence budget: seq_budget is a CUDA int32
+    tensor [B] (see include/lf_decode.h)."""
+    import torch
+    bf = torch.bfloat16
+    cshape = (h.B, h.Hkv, budget, h.D)
+    _check(load_library().lf_decode_step_ragged(
+        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
+        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"), sink, window,
+        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out"),
+        _ptr(evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step_ragged")
+
+
+def lf_decode_attention_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
+                               seq_budget, out) -> None:
+    import torch
+    bf = torch.bfloat16
+    cshape = (h.B, h.Hkv, budget, h.D)
+    _check(load_library().lf_decode_attention_ragged(
+        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
+        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
+        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention_ragged")
 
 
 def lf_decode_step_noalloc(q, k_new, v_new, kcache, vcache, pos, budget: int, sink: int,

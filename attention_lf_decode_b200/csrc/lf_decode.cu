@@ -81,6 +81,10 @@ struct Params {
   float* out;
   int32_t* evicted;
   int* status;
+  const int32_t* seq_budget;  // [B] per-sequence budgets, or null (every row uses all slots)
+  unsigned int* grab;         // row counter of the dynamic schedule (zero between launches)
+  int dyn;                    // rows are taken from `grab` instead of a static stride
+  int hkv;
   int rows;
   int budget;
   int chunk;
@@ -112,6 +116,11 @@ struct Local {
   uint64_t xa[2];        // cluster exchange 1 received: max / sum / positions / partial output
   uint64_t xb[2];        // cluster exchange 2 received: candidate keys
   uint64_t xc[2];        // cluster exchange 3 received: fp64 rescoring
+  uint64_t grab_bar[2];  // dynamic schedule: the row rank 0 took for this CTA landed
+  int grab_val[2];       // dynamic schedule: that row (-1: none left)
+  int row_id[2];         // row of a metadata buffer (-1: no more rows)
+  int row_nb[2];         // its budget (slots 0 .. nb - 1 exist)
+  int row_bad[2];        // its budget was out of range (clamped, nothing written)
   float s_new[GP];
   float Mg[GP], Lg[GP];
   float cf[kMaxSplit][GP];
@@ -346,10 +355,19 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
   const int ncl = static_cast<int>(gridDim.y), cid = static_cast<int>(blockIdx.y);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = p.budget, chunk = p.chunk, nst = p.nstages;
-  const int slot0 = rank * chunk;
-  const int nvalid = max(0, min(chunk, N - slot0));
-  const int ntiles = (nvalid + T - 1) / T;
-  const int niter = cid < p.rows ? (p.rows - cid + ncl - 1) / ncl : 0;
+  // A row's slots 0 .. nb - 1 are split evenly over the cluster (the shared
+  // buffers are sized for nb = N): this CTA owns nvalid slots from slot0.
+  struct RowGeo {
+    int slot0, nvalid, ntiles;
+  };
+  auto row_geo = [&](int nb) {
+    RowGeo g;
+    const int ch = ((nb + S - 1) / S + 3) & ~3;
+    g.slot0 = rank * ch;
+    g.nvalid = max(0, min(ch, nb - g.slot0));
+    g.ntiles = (g.nvalid + T - 1) / T;
+    return g;
+  };
 
   extern __shared__ __align__(128) unsigned char smem[];
   const typename Geo::Layout L = Geo::layout(chunk, nst);
@@ -401,6 +419,7 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
       mbar_init(&loc.xa[b], 1);  // the receiver's own expect-tx arrival + bytes
       mbar_init(&loc.xb[b], 1);
       mbar_init(&loc.xc[b], 1);
+      mbar_init(&loc.grab_bar[b], 1);
     }
     loc.err = 0;
     fence_mbar_init();
@@ -415,21 +434,68 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
 
   if (warp == CW) {
     // ================================================================ producer
-    auto issue_meta = [&](int it) {
-      const int row = cid + it * ncl;
+    // The row of iteration it: a static stride over the rows, or (dynamic
+    // schedule) the next row of a global counter, taken by rank 0 and sent
+    // to every CTA of the cluster.  Every cluster takes rows until it gets
+    // none, so a launch takes exactly rows + clusters values; the one that
+    // takes the last value resets the counter for the next launch.
+    auto next_row = [&](int it) -> int {
+      if (!p.dyn) {
+        const int r = cid + it * ncl;
+        return r < p.rows ? r : -1;
+      }
+      const int b = it & 1;
+      int r = -1;
+      if (lane == 0) {
+        if (rank == 0) {
+          const unsigned g = atomicAdd(p.grab, 1u);
+          const int rr = g < unsigned(p.rows) ? int(g) : -1;
+          if (g == unsigned(p.rows + ncl - 1)) atomicExch(p.grab, 0u);
+          const uint32_t va = smem_addr(&loc.grab_val[b]), ba = smem_addr(&loc.grab_bar[b]);
+          for (int q = 0; q < S; ++q)
+            st_async_b32(map_rank_addr(va, q), uint32_t(rr), map_rank_addr(ba, q));
+        }
+        mbar_arrive_expect_tx(&loc.grab_bar[b], 4u);
+        wait_cl(&loc.grab_bar[b], uint32_t((it >> 1) & 1));
+        r = loc.grab_val[b];
+      }
+      return __shfl_sync(0xffffffffu, r, 0);
+    };
+    // load the metadata of iteration it's row (or mark the end of the rows)
+    auto issue_meta = [&](int it, int row) {
       const int b = it & 1;
       if (it >= 2 && lane == 0) wait_cta(&loc.row_free[b], uint32_t((it >> 1) & 1) ^ 1u);
       __syncwarp();
+      if (row < 0) {
+        if (lane == 0) {
+          loc.row_id[b] = -1;
+          mbar_arrive(&loc.row_full[b]);
+        }
+        __syncwarp();
+        return;
+      }
+      int nb = N, bad = 0;
+      if (p.seq_budget) {
+        nb = p.seq_budget[row / p.hkv];
+        bad = (nb < 1 || nb > N) ? 1 : 0;
+        nb = min(max(nb, 1), N);
+      }
+      const RowGeo rg = row_geo(nb);
+      const int slot0 = rg.slot0, nvalid = rg.nvalid;
       int* ps = pos_buf(b);
       const int32_t* pg = p.pos + size_t(row) * N + slot0;
       const uint32_t mbytes = uint32_t(G * D * 2 + 2 * D * 2);
-      if (!p.pos_bulk) {
+      const bool bulk = p.pos_bulk && (nvalid & 3) == 0;
+      if (!bulk) {
         for (int j = lane; j < nvalid; j += 32) ps[j] = pg[j];
         __syncwarp();
         __threadfence_block();
       }
       if (lane == 0) {
-        const uint32_t pbytes = p.pos_bulk ? uint32_t(nvalid) * 4 : 0u;
+        loc.row_id[b] = row;
+        loc.row_nb[b] = nb;
+        loc.row_bad[b] = bad;
+        const uint32_t pbytes = bulk ? uint32_t(nvalid) * 4 : 0u;
         mbar_arrive_expect_tx(&loc.row_full[b], mbytes + pbytes);
         if (pbytes) bulk_copy_g2s(ps, pg, pbytes, &loc.row_full[b]);
         bulk_copy_g2s(q_buf(b), p.q + size_t(row) * G * D, G * D * 2, &loc.row_full[b]);
@@ -438,11 +504,12 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
       }
       __syncwarp();
     };
-    auto issue_tiles = [&](int it, int phase) {
-      const int row = cid + it * ncl;
+    auto issue_tiles = [&](int it, int row, int phase) {
       const int* ps = pos_buf(it & 1);
+      const RowGeo rg = row_geo(loc.row_nb[it & 1]);
+      const int nvalid = rg.nvalid, ntiles = rg.ntiles;
       const uint16_t* base =
-          (phase == 0 ? p.kcache : p.vcache) + (size_t(row) * N + slot0) * D;
+          (phase == 0 ? p.kcache : p.vcache) + (size_t(row) * N + rg.slot0) * D;
       for (int tile = 0; tile < ntiles; ++tile) {
         if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
         const int s = stg;
@@ -463,12 +530,15 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
         }
       }
     };
-    if (niter > 0) issue_meta(0);
-    for (int it = 0; it < niter; ++it) {
+    int row = next_row(0);
+    issue_meta(0, row);
+    for (int it = 0; row >= 0; ++it) {
       wait_cta(&loc.row_full[it & 1], uint32_t((it >> 1) & 1));
-      issue_tiles(it, 0);
-      if (it + 1 < niter) issue_meta(it + 1);
-      issue_tiles(it, 1);
+      issue_tiles(it, row, 0);
+      const int nrow = next_row(it + 1);
+      issue_meta(it + 1, nrow);
+      issue_tiles(it, row, 1);
+      row = nrow;
     }
   } else {
     // ================================================================ consumers
@@ -487,12 +557,16 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
     const int eh = lane % GP;   // head of this lane in the probability pass
     uint32_t xc_uses0 = 0, xc_uses1 = 0;
 
-    for (int it = 0; it < niter; ++it) {
-      const int row = cid + it * ncl;
+    for (int it = 0;; ++it) {
       const int b = it & 1;
       const uint32_t bpar = uint32_t((it >> 1) & 1);
       const int* ps = pos_buf(b);
       wait_cta(&loc.row_full[b], bpar);
+      const int row = loc.row_id[b];
+      if (row < 0) break;
+      const RowGeo rg = row_geo(loc.row_nb[b]);
+      const int slot0 = rg.slot0, nvalid = rg.nvalid, ntiles = rg.ntiles;
+      if (tid == 0 && rank == 0 && loc.row_bad[b]) atomicOr(p.status, LF_STATUS_BAD_SEQ_BUDGET);
 
       // query heads of the group, fp32, pre-scaled, in this lane's head order
       float2 qp[GP][DPL / 2];
@@ -1030,7 +1104,7 @@ __global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kern
         // -------------------------------------------- in-place eviction
         if (rank == 0) {
           int e, ev;
-          if (loc.g_err || loc.err) {
+          if (loc.g_err || loc.err || loc.row_bad[b]) {
             e = -1;
             ev = -2;
           } else if (!full_row) {
@@ -1120,7 +1194,8 @@ struct lf_ctx {
   int sm_count;
   int smem_optin;
   int split_override;
-  int* status;  // device status word
+  int* status;          // device status word
+  unsigned int* grab;   // device row counter of the dynamic schedule (after the status word)
   int last_bits;
   int score_mode;  // LF_SCORE_* used by lf_decode_step
   Plan plan[3];    // [kernel mode]
@@ -1281,8 +1356,10 @@ cudaError_t get_plan(lf_ctx* c, int budget, int mode, Plan** out) {
 
 int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                uint16_t* kcache, uint16_t* vcache, int32_t* pos, int budget, int sink,
-               int window, float* out, int32_t* evicted, bool evict) {
+               int window, float* out, int32_t* evicted, bool evict,
+               const int32_t* seq_budget = nullptr) {
   if (!valid_handle(h)) return LF_ENOTINIT;
+  if (seq_budget && (!aligned(seq_budget, 4) || !h->grab)) return LF_EINVAL;
   if (!q || !k_new || !v_new || !kcache || !vcache || !pos || !out) return LF_EINVAL;
   if (evict && !evicted) return LF_EINVAL;
   if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(kcache, 16) ||
@@ -1310,6 +1387,10 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   p.out = out;
   p.evicted = evicted;
   p.status = h->status;
+  p.seq_budget = seq_budget;
+  p.grab = h->grab;
+  p.dyn = seq_budget ? 1 : 0;
+  p.hkv = h->Hkv;
   p.rows = h->B * h->Hkv;
   p.budget = budget;
   p.chunk = pl->chunk;
@@ -1383,11 +1464,13 @@ int lf_init(lf_handle* out, int B, int Hq, int Hkv, int D, int max_budget, void*
   c->split_override = 0;
   c->score_mode = LF_SCORE_MEAN_PROB;
   c->magic = kMagic;
-  if (cudaMalloc(&c->status, sizeof(int)) != cudaSuccess) {
+  // the status word, then the row counter of the dynamic schedule
+  if (cudaMalloc(&c->status, 2 * sizeof(int)) != cudaSuccess) {
     free(c);
     return LF_ECUDA;
   }
-  if (cudaMemset(c->status, 0, sizeof(int)) != cudaSuccess) {
+  c->grab = reinterpret_cast<unsigned int*>(c->status + 1);
+  if (cudaMemset(c->status, 0, 2 * sizeof(int)) != cudaSuccess) {
     cudaFree(c->status);
     free(c);
     return LF_ECUDA;
@@ -1467,6 +1550,25 @@ int lf_decode_attention(lf_handle h, const uint16_t* q, const uint16_t* k_new,
                     nullptr, false);
 }
 
+int lf_decode_step_ragged(lf_handle h, const uint16_t* q, const uint16_t* k_new,
+                          const uint16_t* v_new, uint16_t* kcache, uint16_t* vcache,
+                          int32_t* pos, int budget, const int32_t* seq_budget, int sink,
+                          int window, float* out, int32_t* evicted_idx) {
+  if (!seq_budget) return LF_EINVAL;
+  return run_decode(h, q, k_new, v_new, kcache, vcache, pos, budget, sink, window, out,
+                    evicted_idx, true, seq_budget);
+}
+
+int lf_decode_attention_ragged(lf_handle h, const uint16_t* q, const uint16_t* k_new,
+                               const uint16_t* v_new, const uint16_t* kcache,
+                               const uint16_t* vcache, const int32_t* pos, int budget,
+                               const int32_t* seq_budget, float* out) {
+  if (!seq_budget) return LF_EINVAL;
+  return run_decode(h, q, k_new, v_new, const_cast<uint16_t*>(kcache),
+                    const_cast<uint16_t*>(vcache), const_cast<int32_t*>(pos), budget, 0, 1, out,
+                    nullptr, false, seq_budget);
+}
+
 int lf_get_status(lf_handle h) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (cudaStreamSynchronize(h->stream) != cudaSuccess) return LF_ECUDA;
@@ -1474,6 +1576,10 @@ int lf_get_status(lf_handle h) {
   if (cudaMemcpy(&bits, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return LF_ECUDA;
   if (bits != 0 && cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return LF_ECUDA;
+  // a launch whose waits gave up may have left the dynamic schedule's row
+  // counter away from zero
+  if ((bits & LF_STATUS_WAIT_TIMEOUT) && cudaMemset(h->grab, 0, sizeof(unsigned)) != cudaSuccess)
+    return LF_ECUDA;
   h->last_bits = bits;
   return bits ? LF_EDEVICE : LF_OK;
 }

@@ -44,6 +44,7 @@ _T_KNEW = 6
 _T_VNEW = 7
 _T_KNEW_MASK = 8
 _T_AR_INIT = 9
+_T_SEQ_BUDGET = 10
 _PREFILL_KEY = 0  # step_key of prefill draws; decode step s uses s + 1
 
 
@@ -67,6 +68,9 @@ class DecodeConfig:
     new_key_outliers: bool = False
     query_mode: str = "shift"  # "shift" or "ar1"
     ar_rho: float = 0.95
+    # ragged batch: per-sequence budgets drawn uniformly in
+    # [seq_budget_min, budget] (0 = every sequence uses all slots)
+    seq_budget_min: int = 0
 
     @property
     def group(self) -> int:
@@ -106,6 +110,12 @@ CONFIGS = {
                                    head_dim=128, budget=8192, sink=4, window=256,
                                    prefill=8192, steps=16384, seed=4,
                                    query_mode="ar1"),
+    # ragged serving batch: the throughput shape with per-sequence budgets
+    # drawn in [1024, 4096], each sequence's cache full at its own budget
+    "ragged": DecodeConfig("ragged", batch=64, hq=32, hkv=8, head_dim=128,
+                           budget=4096, sink=4, window=128, prefill=4096, steps=256,
+                           seed=5, key_outlier_frac=0.02, key_outlier_mag=4.0,
+                           new_key_outliers=True, seq_budget_min=1024),
     # budget sweep (full caches) and the no-eviction control
     "sweep_n1024": _budget_sweep(1024, 50),
     "sweep_n2048": _budget_sweep(2048, 51),
@@ -221,6 +231,14 @@ class SynthDecode:
             m = _rng(c.seed, sk, _T_KNEW_MASK).random((c.batch, c.hkv)) < c.key_outlier_frac
             kn[m] += np.float32(c.key_outlier_mag) * self.u
         return to_bf16_bits(q), to_bf16_bits(kn), to_bf16_bits(vn)
+
+    def seq_budgets(self) -> Optional[np.ndarray]:
+        """Per-sequence budgets [B] (int32) of a ragged config, else None."""
+        c = self.cfg
+        if not c.seq_budget_min:
+            return None
+        g = _rng(c.seed, _PREFILL_KEY, _T_SEQ_BUDGET)
+        return g.integers(c.seq_budget_min, c.budget + 1, size=c.batch).astype(np.int32)
 
     def iter_steps(self, steps: Optional[int] = None, start: int = 0) -> Iterable:
         n = self.cfg.steps if steps is None else steps

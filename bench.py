@@ -70,13 +70,15 @@ def parse():
 
 # ------------------------------------------------------------------ bytes
 
-def algorithmic_bytes(cfg, filled: int) -> dict:
+def algorithmic_bytes(cfg, filled) -> dict:
     """Bytes one step must move: the K and V of every filled slot once, plus
     every write (fp32 output, the new token's K/V row, its position, the
     evicted index).  q, k_new, v_new and the position table are read too;
-    they are listed apart (under 1%)."""
+    they are listed apart (under 1%).  filled: slots per row, or per
+    sequence ([B], ragged batches)."""
     rows = cfg.batch * cfg.hkv
-    kv_read = rows * filled * cfg.head_dim * 2 * 2
+    kv_read = int(np.sum(np.broadcast_to(np.asarray(filled, np.int64), (cfg.batch,)))) \
+        * cfg.hkv * cfg.head_dim * 2 * 2
     writes = (cfg.batch * cfg.hq * cfg.head_dim * 4 + rows * cfg.head_dim * 2 * 2 + rows * 4
               + rows * 4)
     other_reads = (cfg.batch * cfg.hq * cfg.head_dim * 2 + rows * cfg.head_dim * 2 * 2
@@ -168,7 +170,7 @@ class ClockSampler:
 # ------------------------------------------------------------------ oracle
 
 def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_steps: int,
-                score: str = "mean_prob"):
+                score: str = "mean_prob", seq_budget=None):
     """Time the CPU oracle, as it stands, on sampled batch entries; returns
     (full steps/s extrapolated from rows/s, sample description, steps run)."""
     import oracle
@@ -185,7 +187,8 @@ def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_s
         kn = synth.bf16_bits_to_f64(knb[batch_sel])
         vn = synth.bf16_bits_to_f64(vnb[batch_sel])
         t0 = time.perf_counter()
-        res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window, score=score)
+        res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window, score=score,
+                                 seq_budget=None if seq_budget is None else seq_budget[batch_sel])
         t_total += time.perf_counter() - t0
         K, V, P = res.kcache, res.vcache, res.pos
         n += 1
@@ -259,11 +262,22 @@ def main():
     vn_all = torch.stack([binding.bf16_from_bits(x[2]) for x in inputs])
     out = torch.empty((cfg.batch, cfg.hq, cfg.head_dim), dtype=torch.float32, device=dev)
     ev = torch.empty((cfg.batch, cfg.hkv), dtype=torch.int32, device=dev)
+    # ragged batch: a budget per sequence (the prefill fills every slot; the
+    # slots beyond a sequence's budget are never read)
+    nb_host = gen.seq_budgets()
+    nb_dev = None if nb_host is None else torch.from_numpy(nb_host).to(dev)
+
+    def run(q, kn, vn):
+        if nb_dev is None:
+            binding.lf_decode_step(h, q, kn, vn, kcache, vcache, pos, cfg.budget, cfg.sink,
+                                   cfg.window, out, ev)
+        else:
+            binding.lf_decode_step_ragged(h, q, kn, vn, kcache, vcache, pos, cfg.budget, nb_dev,
+                                          cfg.sink, cfg.window, out, ev)
 
     def step(i):
         j = i % n_inputs
-        binding.lf_decode_step(h, q_all[j], kn_all[j], vn_all[j], kcache, vcache, pos, cfg.budget,
-                               cfg.sink, cfg.window, out, ev)
+        run(q_all[j], kn_all[j], vn_all[j])
 
     # warm-up
     for i in range(max(args.warmup, 3)):
@@ -332,8 +346,7 @@ def main():
             d_q.copy_(hq[j], non_blocking=True)
             d_k.copy_(hk[j], non_blocking=True)
             d_v.copy_(hv[j], non_blocking=True)
-            binding.lf_decode_step(h, d_q, d_k, d_v, kcache, vcache, pos, cfg.budget, cfg.sink,
-                                   cfg.window, out, ev)
+            run(d_q, d_k, d_v)
             h_out.copy_(out, non_blocking=True)
             h_ev.copy_(ev, non_blocking=True)
             stream.synchronize()
@@ -362,7 +375,8 @@ def main():
         if binding.lf_get_status(h) != binding.LF_OK:
             raise RuntimeError("device status after e2e")
 
-    by = algorithmic_bytes(cfg, cfg.budget if cfg.prefill >= cfg.budget else cfg.prefill)
+    filled = min(cfg.budget, cfg.prefill) if nb_host is None else np.minimum(nb_host, cfg.prefill)
+    by = algorithmic_bytes(cfg, filled)
     kern_s = ms_per_step / 1e3  # one launch per step
     achieved = by["algorithmic"] / kern_s / 1e9
     peak, peak_src = measured_peak()
@@ -371,7 +385,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         rate, sample, _ = oracle_rate(cfg, gen, kpre, vpre, args.cpu_seconds, list(range(4)), 64,
-                                      score=args.score)
+                                      score=args.score, seq_budget=nb_host)
         cpu = {"value": rate, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
                "sample": sample}
 
@@ -392,6 +406,10 @@ def main():
             "window": cfg.window, "kv_dtype": "bf16", "accumulate": "f32",
             "parallelism": f"dp{world} (batch per rank, no collective)",
             "split_ctas_per_row": split,
+            "seq_budgets": (None if nb_host is None else
+                            {"min": int(nb_host.min()), "max": int(nb_host.max()),
+                             "mean": float(nb_host.mean()),
+                             "schedule": "dynamic (rows taken from a device counter)"}),
             "score": args.score,
             "l2": "inputs larger than L2: each step reads the 1 GiB K/V cache (L2 is 126 MB)",
             "tokens_per_s": value * cfg.batch,
@@ -428,12 +446,16 @@ def reference_arm(args, cfg, workload, world, rank):
     K, V, P = synth.bf16_bits_to_f64(kc), synth.bf16_bits_to_f64(vc), pos.astype(np.int64)
     budget_s = 150.0
     rows_full = cfg.batch * cfg.hkv
+    nb = gen.seq_budgets()  # ragged batch: the sample's budget and every sequence's
+    nb0 = None if nb is None else nb[:1]
+    # full-step work relative to the sampled rows' (rows of unequal budget)
+    work_ratio = 1.0 if nb is None else float(nb.sum()) / (float(nb[0]) * cfg.batch)
     # calibrate: one row-step
     qb, knb, vnb = gen.step_inputs(0)
     t0 = time.perf_counter()
     oracle.decode_step(K[:, :1], V[:, :1], P[:, :1], synth.bf16_bits_to_f64(qb[:1, :cfg.group]),
                        synth.bf16_bits_to_f64(knb[:1, :1]), synth.bf16_bits_to_f64(vnb[:1, :1]),
-                       cfg.sink, cfg.window)
+                       cfg.sink, cfg.window, seq_budget=nb0)
     t_row = time.perf_counter() - t0
     nsteps = args.warmup + args.steps
     rows_per_step = int(max(1, min(cfg.hkv, budget_s / max(nsteps, 1) / max(t_row, 1e-6))))
@@ -446,15 +468,16 @@ def reference_arm(args, cfg, workload, world, rank):
         vn = synth.bf16_bits_to_f64(vnb[:1, :heads])
         t0 = time.perf_counter()
         res = oracle.decode_step(K[:, :heads], V[:, :heads], P[:, :heads], q, kn, vn,
-                                 cfg.sink, cfg.window, score=args.score)
+                                 cfg.sink, cfg.window, score=args.score, seq_budget=nb0)
         dt = time.perf_counter() - t0
         K[:, :heads], V[:, :heads], P[:, :heads] = res.kcache, res.vcache, res.pos
         if s >= args.warmup:
             t_total += dt
     per_row = t_total / (args.steps * heads)
-    value = 1.0 / (per_row * rows_full)
+    value = 1.0 / (per_row * rows_full * work_ratio)
     sample = (f"each step: oracle on {heads} of {rows_full} rows (batch entry 0), "
-              f"{args.steps} timed steps after {args.warmup} warm-up; steps/s scaled to all rows")
+              f"{args.steps} timed steps after {args.warmup} warm-up; steps/s scaled to all rows"
+              + ("" if nb is None else " in proportion to their budgets"))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,

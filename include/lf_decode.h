@@ -69,6 +69,7 @@ extern "C" {
 /* device status bits, as set by the kernels and returned by lf_status_bits */
 #define LF_STATUS_WAIT_TIMEOUT 1  /* a bounded wait on a shared-memory barrier gave up */
 #define LF_STATUS_NO_CANDIDATE 2  /* full cache but no unprotected slot (corrupt pos table) */
+#define LF_STATUS_BAD_SEQ_BUDGET 4 /* a per-sequence budget outside 1 .. budget (ragged calls) */
 
 /* Eviction scores (lf_set_score) */
 #define LF_SCORE_MEAN_PROB 0  /* probability averaged over the group's query heads (default) */
@@ -137,6 +138,42 @@ LF_API int lf_decode_attention(lf_handle h,
                         const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                         const uint16_t* kcache, const uint16_t* vcache, const int32_t* pos,
                         int budget, float* out);
+
+/* Ragged batch: lf_decode_step with a budget per sequence.
+ * seq_budget: DEVICE int32 [B], 4-byte aligned, owned by the caller and
+ * read by the kernel; batch entry b (all its KV heads) then has the cache
+ * of slots 0 .. seq_budget[b] - 1 alone.  The slots beyond are neither
+ * read (not even for t) nor written, so they may hold anything.  Each
+ * sequence appends while one of its slots is free and evicts once its own
+ * budget is full, exactly as lf_decode_step does for a budget of
+ * seq_budget[b]; rows at different positions and fill levels may share a
+ * batch.  `budget` is still the allocated slots per row (the cache stride)
+ * and bounds every seq_budget[b].
+ * A row's slots are split evenly over the CTAs of its cluster, and the
+ * clusters take rows from a counter in the handle's device memory as they
+ * finish the previous ones (a dynamic schedule: work per row follows
+ * seq_budget[b]).  Calls on one handle must therefore not run concurrently.
+ * Device-side checks: a seq_budget[b] outside 1 .. budget sets
+ * LF_STATUS_BAD_SEQ_BUDGET; its rows get out computed over the clamped
+ * budget, evicted = -2, and no cache write.  A full sequence with
+ * seq_budget[b] <= sink + window has no candidate (LF_STATUS_NO_CANDIDATE,
+ * evicted = -2).  Host checks as lf_decode_step, plus seq_budget non-null
+ * and aligned (else LF_EINVAL).  Follows the handle's score (lf_set_score).
+ * The pages do not treat ragged batches; this is the serving-batch form of
+ * the same per-row step. */
+LF_API int lf_decode_step_ragged(lf_handle h,
+                   const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                   uint16_t* kcache, uint16_t* vcache, int32_t* pos,
+                   int budget, const int32_t* seq_budget, int sink, int window,
+                   float* out, int32_t* evicted_idx);
+
+/* lf_decode_attention with a budget per sequence (seq_budget as in
+ * lf_decode_step_ragged): attention over each sequence's filled slots
+ * among 0 .. seq_budget[b] - 1 plus the new token; only out is written. */
+LF_API int lf_decode_attention_ragged(lf_handle h,
+                        const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                        const uint16_t* kcache, const uint16_t* vcache, const int32_t* pos,
+                        int budget, const int32_t* seq_budget, float* out);
 
 /* Eviction score used by later lf_decode_step calls on this handle.
  *   LF_SCORE_MEAN_PROB (default): score_j as documented for lf_decode_step.
