@@ -28,7 +28,8 @@ LF_SCORE_MEAN_PROB = 0
 LF_SCORE_ALPHA_L1V = 1
 
 EXPORTS = ("lf_init", "lf_set_stream", "lf_prefill_cache", "lf_decode_step",
-           "lf_decode_attention", "lf_decode_step_ragged", "lf_decode_attention_ragged", "lf_set_split", "lf_get_split", "lf_set_score",
+           "lf_decode_attention", "lf_decode_step_ragged", "lf_decode_attention_ragged",
+           "lf_prefill_cache_fp8", "lf_decode_step_fp8", "lf_decode_attention_fp8", "lf_set_split", "lf_get_split", "lf_set_score",
            "lf_get_score", "lf_get_status",
            "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version",
            "lf_decode_step_noalloc")
@@ -52,7 +53,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         raise FileNotFoundError(
             f"{path} is missing: build it with `python -m attention_lf_decode_b200.build`")
     lib = ctypes.CDLL(path)
-    P, I, VP = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+    P, I, VP, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_float
     sig = {
         "lf_init": ([ctypes.POINTER(P), I, I, I, I, I, VP], I),
         "lf_set_stream": ([P, VP], I),
@@ -61,6 +62,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lf_decode_attention": ([P, VP, VP, VP, VP, VP, VP, I, VP], I),
         "lf_decode_step_ragged": ([P, VP, VP, VP, VP, VP, VP, I, VP, I, I, VP, VP], I),
         "lf_decode_attention_ragged": ([P, VP, VP, VP, VP, VP, VP, I, VP, VP], I),
+        "lf_prefill_cache_fp8": ([P, VP, VP, I, VP, VP, VP, I, F, F], I),
+        "lf_decode_step_fp8": ([P, VP, VP, VP, VP, VP, VP, I, VP, I, I, F, F, VP, VP], I),
+        "lf_decode_attention_fp8": ([P, VP, VP, VP, VP, VP, VP, I, VP, F, F, VP], I),
         "lf_set_split": ([P, I], I),
         "lf_get_split": ([P, I], I),
         "lf_set_score": ([P, I], I),
@@ -233,6 +237,54 @@ def lf_decode_attention_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, 
         _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
         _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
         _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention_ragged")
+
+
+def lf_prefill_cache_fp8(h: Handle, k, v, n: int, kcache, vcache, pos, budget: int,
+                         k_scale: float, v_scale: float) -> None:
+    """Prefill an E4M3 cache (kcache / vcache: CUDA uint8 [B, Hkv, budget, D])
+    from bf16 prompt K/V [B, Hkv, n, D]."""
+    import torch
+    bf, u8 = torch.bfloat16, torch.uint8
+    cshape = (h.B, h.Hkv, budget, h.D)
+    kp = _ptr(k, bf, (h.B, h.Hkv, n, h.D), "k") if n > 0 else None
+    vp = _ptr(v, bf, (h.B, h.Hkv, n, h.D), "v") if n > 0 else None
+    _check(load_library().lf_prefill_cache_fp8(
+        h.ptr, kp, vp, n, _ptr(kcache, u8, cshape, "kcache"), _ptr(vcache, u8, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget, k_scale, v_scale),
+        "lf_prefill_cache_fp8")
+
+
+def lf_decode_step_fp8(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int, sink: int,
+                       window: int, k_scale: float, v_scale: float, out, evicted_idx,
+                       seq_budget=None) -> None:
+    """The decode step on an E4M3 cache (see include/lf_decode.h)."""
+    import torch
+    bf, u8 = torch.bfloat16, torch.uint8
+    cshape = (h.B, h.Hkv, budget, h.D)
+    _check(load_library().lf_decode_step_fp8(
+        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
+        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _ptr(kcache, u8, cshape, "kcache"), _ptr(vcache, u8, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        None if seq_budget is None else _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
+        sink, window, k_scale, v_scale,
+        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out"),
+        _ptr(evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step_fp8")
+
+
+def lf_decode_attention_fp8(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
+                            k_scale: float, v_scale: float, out, seq_budget=None) -> None:
+    import torch
+    bf, u8 = torch.bfloat16, torch.uint8
+    cshape = (h.B, h.Hkv, budget, h.D)
+    _check(load_library().lf_decode_attention_fp8(
+        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
+        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _ptr(kcache, u8, cshape, "kcache"), _ptr(vcache, u8, cshape, "vcache"),
+        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        None if seq_budget is None else _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
+        k_scale, v_scale, _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")),
+        "lf_decode_attention_fp8")
 
 
 def lf_decode_step_noalloc(q, k_new, v_new, kcache, vcache, pos, budget: int, sink: int,

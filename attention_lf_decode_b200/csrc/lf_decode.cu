@@ -1,1152 +1,10 @@
-// B200 (sm_100a) LongFlow fused decode step: single-query GQA attention,
-// the zero-history / zero-cost importance score taken from the same softmax,
-// and the in-place eviction of the least important unprotected slot, all in
-// ONE launch.  The C ABI is declared in include/lf_decode.h.
-//
-// Method: "LongFlow: Efficient KV Cache Compression for Reasoning Models"
-// (gist.science summary), §2A "Principios de Diseño", §2B "Derivación de la
-// Métrica de Importancia", §2C "Implementación de Alto Rendimiento"; blog
-// page "Долгая память: Оптимизация кэша для сложных рассуждений", section
-// "Оптимизированная Реализация с Объединенными Ядрами" (attention output
-// and score produced in one pass over KV blocks and a mask streamed from HBM
-// into on-chip memory).
-//
-// Design.  One row = one (batch, KV head) pair; its K and V slabs are each
-// [budget, D] bf16, contiguous.
-//   * Persistent thread-block clusters: a cluster of S CTAs owns a row at a
-//     time and splits its slots into S chunks (flash-decoding split); the
-//     cluster then moves on to row + (number of clusters).  Each CTA has 8
-//     consumer warps and 1 producer warp.
-//   * The producer streams the chunk's K tiles, then its V tiles (16 KB each,
-//     contiguous) with 1-D bulk async copies into an mbarrier-guarded ring,
-//     without a pause between rows: while the consumers finish one row, the
-//     next row's position table, query heads and new K/V are already loaded
-//     and its first tiles are in flight.  Tiles whose slots are all free are
-//     never loaded.  No multicast: every CTA fetches its own tiles.
-//   * K phase: 8 lanes per slot, 16-byte conflict-free shared loads, packed
-//     fp32x2 FMAs against the pre-scaled query heads held in registers in a
-//     per-lane head order that lets the 8-lane reduce-scatter run without
-//     selects.  Logits (log2 domain) stay in shared memory: the exact
-//     normalised probabilities need the row-wide max and sum, which only
-//     exist once every CTA of the cluster is done.
-//   * V phase: p = 2^(s - m_cta) in place, o += p * v with 8 dims per lane
-//     and packed FMAs.
-//   * Cluster exchange through distributed shared memory, signalled by
-//     remote mbarrier arrivals (release / acquire at cluster scope) into
-//     per-row-parity buffers, so no whole-cluster barrier stops the
-//     producer: row max / sum per head, newest position, lowest free slot;
-//     then each CTA scores its own slots (exact normalised probability
-//     averaged over the group's heads), reduces packed (fp32 score bits << 32
-//     | slot) keys to the two lowest, and combines its share of the output.
-//   * Near ties (two lowest scores within a relative 1e-4) are rescored in
-//     fp64 from the cache, so the choice follows the exact ranking.
-//   * CTA rank 0 writes k_new / v_new / t into the chosen slot after the key
-//     exchange, which every CTA enters only after its last read of the row.
-#include <cooperative_groups.h>
-#include <cuda_runtime.h>
-#include <limits.h>
-#include <math.h>
-#include <stdint.h>
-#include <stdio.h>
-#include <stdlib.h>
-#include <string.h>
-
-#include <mutex>
-
-#include "lf_decode.h"
-#include "lf_ptx.cuh"
-
-namespace cg = cooperative_groups;
+// B200 (sm_100a) LongFlow fused decode step: the C ABI declared in
+// include/lf_decode.h (handles, argument checks, launch planning cache,
+// dispatch to the compiled kernel variants), the prefill kernels and the
+// allocation-free entry point.  The fused kernel itself is in lf_kernel.cuh.
+#include "lf_kernel.cuh"
 
 namespace lf {
-
-constexpr int kMaxCW = 11;                  // most consumer warps of any variant
-constexpr int kMaxStages = 4;
-constexpr int kMinStages = 2;
-constexpr int kMaxSplit = 16;
-constexpr int kMaxG = 8;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
-constexpr float kTieRel = 1e-4f;                   // near-tie band rescored in fp64
-constexpr unsigned long long kNoKey = ~0ull;
-constexpr int kBarConsumers = 1;                   // named barrier of the consumer warps
-constexpr int kAttendOnly = 0, kEvictMeanProb = 1, kEvictAlphaL1V = 2;  // kernel modes
-
-struct Params {
-  const uint16_t* q;
-  const uint16_t* k_new;
-  const uint16_t* v_new;
-  uint16_t* kcache;
-  uint16_t* vcache;
-  int32_t* pos;
-  float* out;
-  int32_t* evicted;
-  int* status;
-  const int32_t* seq_budget;  // [B] per-sequence budgets, or null (every row uses all slots)
-  unsigned int* grab;         // row counter of the dynamic schedule (zero between launches)
-  int dyn;                    // rows are taken from `grab` instead of a static stride
-  int hkv;
-  int rows;
-  int budget;
-  int chunk;
-  int sink;
-  int window;
-  int nstages;
-  int pos_bulk;      // position rows may be bulk-copied (16-byte aligned)
-  float qscale2;     // log2(e) / sqrt(D)
-  double qscale2_64;
-};
-
-// What the CTAs of a cluster send each other about one row (one copy per
-// row parity, in every CTA).  Each CTA writes its own entries [rank] into
-// every CTA's copy with st.async; the receiver's mbarrier counts the bytes.
-template <int GP>
-struct Rx {
-  uint32_t sc[kMaxSplit][2 * GP + 4];     // per sender: m[GP], l[GP], maxpos, first_free, err
-  unsigned long long key[kMaxSplit][2];   // per sender: two lowest candidate keys
-  unsigned long long ref[kMaxSplit][2];   // per sender: fp64 rescoring (score bits, slot)
-};
-
-// CTA-local barriers and scalars.
-template <int GP>
-struct Local {
-  uint64_t full[kMaxStages];
-  uint64_t empty[kMaxStages];
-  uint64_t row_full[2];  // row metadata (positions, q, k_new, v_new) landed
-  uint64_t row_free[2];  // consumers are done with a metadata buffer
-  uint64_t xa[2];        // cluster exchange 1 received: max / sum / positions / partial output
-  uint64_t xb[2];        // cluster exchange 2 received: candidate keys
-  uint64_t xc[2];        // cluster exchange 3 received: fp64 rescoring
-  uint64_t grab_bar[2];  // dynamic schedule: the row rank 0 took for this CTA landed
-  int grab_val[2];       // dynamic schedule: that row (-1: none left)
-  int row_id[2];         // row of a metadata buffer (-1: no more rows)
-  int row_nb[2];         // its budget (slots 0 .. nb - 1 exist)
-  int row_bad[2];        // its budget was out of range (clamped, nothing written)
-  float s_new[GP];
-  float Mg[GP], Lg[GP];
-  float cf[kMaxSplit][GP];
-  float wmax[kMaxCW][GP];
-  float wsum[kMaxCW][GP];
-  int wpmax[kMaxCW], wpfree[kMaxCW];
-  unsigned long long wk1[kMaxCW], wk2[kMaxCW];
-  double wref[kMaxCW];
-  int wrefs[kMaxCW];
-  unsigned long long g_key1;
-  int g_t, g_free, g_err, g_refine, g_slot;
-  int err;
-};
-
-__host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
-__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
-
-template <int D, int G>
-struct Geometry {
-  static constexpr int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
-  // Consumer warps.  One SM runs one CTA; with 12 warps a scheduler holds 3,
-  // which leaves 168 registers per thread: 11 consumers + the producer.  The
-  // 8-head variants need more registers per thread and keep 8 consumers.
-  static constexpr int CW = GP >= 8 ? 8 : 11;
-  static constexpr int kConsumers = CW * 32;
-  static constexpr int kThreads = kConsumers + 32;  // + 1 producer warp
-  // Bytes per ring stage: large tiles amortise the per-tile work.  A tile
-  // holds 16 slots per consumer warp (176 at D = 128) for the small groups,
-  // 32 KB for the 8-head variants (which keep twice the probabilities).
-  static constexpr int kTile = GP >= 8 ? 32768 : CW * 16 * 2 * 128;
-  static constexpr int T = kTile / (2 * D);        // slots per tile
-  static constexpr int CPL = D / 64;               // K phase: 16-byte chunks per lane
-  static constexpr int DPL = CPL * 8;              // K phase: dims per lane
-  static constexpr int GROUPS = T / 4;             // K phase: 4-slot groups per tile
-  static constexpr int GPW = GROUPS / CW;          // K phase: groups per warp per tile
-  // K phase: groups computed together (more in flight hides latency; the
-  // 8-head variants hold twice the query registers, so they take fewer)
-  static constexpr int KU = GP >= 8 ? 1 : (GPW < 4 ? GPW : 4);
-  static constexpr int VL = D / 8;                 // V phase: lanes per slot (8 dims each)
-  static constexpr int SPV = 32 / VL;              // V phase: slots per warp pass
-  static constexpr int TPW = T / CW;               // V phase: slots per warp per tile
-  static constexpr int VU = TPW / SPV;             // V phase: slot passes unrolled together
-  static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
-  static constexpr size_t kMetaStride = align128(size_t(G) * D * 2 + 2 * D * 2);
-  // per parity: this CTA's slice of every CTA's partial output, then Rx
-  static constexpr size_t kPubStride = align128(size_t(G) * D * 4) + align128(sizeof(Rx<GP>));
-  static_assert(GROUPS % CW == 0 && T % CW == 0 && TPW % SPV == 0 && CW <= kMaxCW, "tile split");
-
-  struct Layout {
-    size_t ring, pl, pos, red, pp, meta, pub, loc, total;
-  };
-  __host__ __device__ static Layout layout(int chunk, int nst) {
-    Layout L;
-    size_t o = 0;
-    L.ring = o; o = align128(o + size_t(nst) * kTile);
-    // logits of whole tiles: the last tile of a chunk may be partial
-    L.pl = o;   o = align128(o + size_t((chunk + T - 1) / T * T) * GP * 4);
-    L.pos = o;  o = align128(o + size_t(2) * chunk * 4);
-    L.red = o;  o = align128(o + size_t(CW) * G * D * 4);
-    L.pp = o;   o = align128(o + size_t(CW) * TPW * GP * 8);
-    L.meta = o; o = align128(o + 2 * kMetaStride);
-    L.pub = o;  o = align128(o + 2 * kPubStride);
-    L.loc = o;  o = align128(o + sizeof(Local<GP>));
-    L.total = o;
-    return L;
-  }
-};
-
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-// 2^x on the SFU (flushes results below 2^-126 to zero; such probabilities
-// change no output, and equal zero scores are settled by the fp64 rescoring)
-__device__ __forceinline__ float ex2_ftz(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ double bf16_to_f64(uint16_t b) {
-  return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16));
-}
-
-__device__ __forceinline__ void flag_error(int* err_smem, int* status) {
-  *err_smem = 1;
-  atomicOr(status, LF_STATUS_WAIT_TIMEOUT);
-}
-
-// keep the two smallest keys
-__device__ __forceinline__ void top2_insert(unsigned long long& k1, unsigned long long& k2,
-                                            unsigned long long k) {
-  if (k < k1) {
-    k2 = k1;
-    k1 = k;
-  } else if (k < k2) {
-    k2 = k;
-  }
-}
-__device__ __forceinline__ void top2_merge(unsigned long long& k1, unsigned long long& k2,
-                                           unsigned long long o1, unsigned long long o2) {
-  const unsigned long long lo = k1 < o1 ? k1 : o1;
-  const unsigned long long hi = k1 < o1 ? o1 : k1;
-  const unsigned long long s2 = k2 < o2 ? k2 : o2;
-  k1 = lo;
-  k2 = hi < s2 ? hi : s2;
-}
-__device__ __forceinline__ void top2_warp(unsigned long long& k1, unsigned long long& k2) {
-#pragma unroll
-  for (int m = 16; m > 0; m >>= 1) {
-    const unsigned long long o1 = __shfl_xor_sync(0xffffffffu, k1, m);
-    const unsigned long long o2 = __shfl_xor_sync(0xffffffffu, k2, m);
-    top2_merge(k1, k2, o1, o2);
-  }
-}
-
-// Any slot of tile `tile` (chunk-local) filled / every slot filled?  Warp-uniform.
-template <int T>
-__device__ __forceinline__ bool tile_filled(const int* ps, int tile, int nvalid, int lane) {
-  bool any = false;
-#pragma unroll
-  for (int k = 0; k < T / 32; ++k) {
-    const int j = tile * T + k * 32 + lane;
-    any |= (j < nvalid) && (ps[j] >= 0);
-  }
-  return __any_sync(0xffffffffu, any);
-}
-template <int T>
-__device__ __forceinline__ bool tile_full(const int* ps, int tile, int nvalid, int lane) {
-  bool all = true;
-#pragma unroll
-  for (int k = 0; k < T / 32; ++k) {
-    const int j = tile * T + k * 32 + lane;
-    all &= (j < nvalid) && (ps[j] >= 0);
-  }
-  return __all_sync(0xffffffffu, all);
-}
-
-// ---- cluster-scope mbarrier signalling (remote arrive, acquire wait)
-__device__ __forceinline__ uint32_t map_rank(const void* p, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ uint32_t map_rank_addr(uint32_t smem_address, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_address), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-__device__ __forceinline__ void fence_cluster() {
-  asm volatile("fence.acq_rel.cluster;" ::: "memory");
-}
-// Non-blocking poll: a waiter suspended inside try_wait is not woken
-// promptly by arrivals from other CTAs, so cluster-level waits poll.
-__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-__device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
-  if (try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (try_wait_cluster(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-
-// Asynchronous stores into the shared memory of a CTA of the cluster (this
-// one included), completing `bytes` on that CTA's mbarrier.  No release
-// fence is involved: a waiter that sees the mbarrier phase complete sees the
-// data.  Addresses are shared::cluster addresses from map_rank().
-__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr),
-               "r"(v), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void st_async_b64(uint32_t addr, unsigned long long v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(addr),
-               "l"(v), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
-      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
-      : "memory");
-}
-
-// One reduce-scatter step over the 8 lanes of a slot.  The lane keeps the
-// first C/2 partial sums and sends the rest; because every lane holds its
-// heads in the order k ^ perm(lane), the partner's second half holds exactly
-// the heads of this lane's first half, so no select is needed.  With C == 1
-// it is a butterfly step.
-template <int C, int MASK>
-__device__ __forceinline__ void rs_step(float (&a)[kMaxG]) {
-  if constexpr (C > 1) {
-#pragma unroll
-    for (int i = 0; i < C / 2; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[C / 2 + i], MASK);
-  } else {
-    a[0] += __shfl_xor_sync(0xffffffffu, a[0], MASK);
-  }
-}
-
-// MODE: kAttendOnly (attention, nothing scored or written), kEvictMeanProb
-// (evict the lowest head-averaged probability) or kEvictAlphaL1V (evict the
-// lowest head-averaged probability times the L1 norm of the slot's value).
-template <int D, int G, int MODE>
-__global__ void __launch_bounds__(Geometry<D, G>::kThreads, 1) fused_decode_kernel(const Params p) {
-  using Geo = Geometry<D, G>;
-  constexpr bool EVICT = MODE != kAttendOnly;
-  constexpr bool L1V = MODE == kEvictAlphaL1V;
-  constexpr int CW = Geo::CW, kConsumers = Geo::kConsumers;
-  constexpr int T = Geo::T, GP = Geo::GP, CPL = Geo::CPL, DPL = Geo::DPL;
-  constexpr int GPW = Geo::GPW, KU = Geo::KU, VU = Geo::VU, VL = Geo::VL, SPV = Geo::SPV,
-                TPW = Geo::TPW;
-  static_assert(G >= 1 && G <= kMaxG, "group size");
-  static_assert(D == 64 || D == 128, "head dim");
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int S = static_cast<int>(cluster.num_blocks());
-  const int ncl = static_cast<int>(gridDim.y), cid = static_cast<int>(blockIdx.y);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int N = p.budget, chunk = p.chunk, nst = p.nstages;
-  // A row's slots 0 .. nb - 1 are split evenly over the cluster (the shared
-  // buffers are sized for nb = N): this CTA owns nvalid slots from slot0.
-  struct RowGeo {
-    int slot0, nvalid, ntiles;
-  };
-  auto row_geo = [&](int nb) {
-    RowGeo g;
-    const int ch = ((nb + S - 1) / S + 3) & ~3;
-    g.slot0 = rank * ch;
-    g.nvalid = max(0, min(ch, nb - g.slot0));
-    g.ntiles = (g.nvalid + T - 1) / T;
-    return g;
-  };
-
-  extern __shared__ __align__(128) unsigned char smem[];
-  const typename Geo::Layout L = Geo::layout(chunk, nst);
-  unsigned char* ring = smem + L.ring;
-  float* pl = reinterpret_cast<float*>(smem + L.pl);     // [chunk][GP] logits, then p
-  int* pos0 = reinterpret_cast<int*>(smem + L.pos);      // [2][chunk]
-  float* red = reinterpret_cast<float*>(smem + L.red);   // [CW][G][D]
-  float2* pp = reinterpret_cast<float2*>(smem + L.pp);   // [CW][TPW][GP] (p, p) pairs
-  unsigned char* meta0 = smem + L.meta;                  // [2] {q[G][D], k_new[D], v_new[D]}
-  unsigned char* pub0 = smem + L.pub;                    // [2] {xo[G][D], Pub}
-  Local<GP>& loc = *reinterpret_cast<Local<GP>*>(smem + L.loc);
-
-  // Bounded waits.  After a first wait has given up (error flagged), later
-  // waits only poll once, so a failed launch ends quickly instead of waiting
-  // the full limit at every barrier.
-  auto wait_cta = [&](uint64_t* bar, uint32_t par) {
-    if (*reinterpret_cast<volatile int*>(&loc.err)) {
-      (void)mbar_try_wait(bar, par);
-      return;
-    }
-    if (!mbar_wait_bounded(bar, par, kWaitLimitNs)) flag_error(&loc.err, p.status);
-  };
-  auto wait_cl = [&](uint64_t* bar, uint32_t par) {
-    if (*reinterpret_cast<volatile int*>(&loc.err)) {
-      (void)try_wait_cluster(bar, par);
-      return;
-    }
-    if (!wait_cluster_bounded(bar, par)) flag_error(&loc.err, p.status);
-  };
-  auto pos_buf = [&](int b) { return pos0 + b * chunk; };
-  auto q_buf = [&](int b) { return reinterpret_cast<uint16_t*>(meta0 + b * Geo::kMetaStride); };
-  auto kn_buf = [&](int b) { return q_buf(b) + G * D; };
-  auto vn_buf = [&](int b) { return q_buf(b) + G * D + D; };
-  // [S][E / S] partial outputs of every sender for this CTA's output slice
-  auto rxo_buf = [&](int b) { return reinterpret_cast<float*>(pub0 + b * Geo::kPubStride); };
-  auto rx_buf = [&](int b) {
-    return reinterpret_cast<Rx<GP>*>(pub0 + b * Geo::kPubStride + align128(size_t(G) * D * 4));
-  };
-
-  if (tid == 0) {
-    for (int s = 0; s < nst; ++s) {
-      mbar_init(&loc.full[s], 1);
-      mbar_init(&loc.empty[s], CW);
-    }
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&loc.row_full[b], 1);
-      mbar_init(&loc.row_free[b], 1);
-      mbar_init(&loc.xa[b], 1);  // the receiver's own expect-tx arrival + bytes
-      mbar_init(&loc.xb[b], 1);
-      mbar_init(&loc.xc[b], 1);
-      mbar_init(&loc.grab_bar[b], 1);
-    }
-    loc.err = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  cluster.sync();  // every CTA's barriers exist before the first remote arrival
-
-  // ring position: tiles issued (producer) or consumed (consumers) so far, and
-  // the stage / phase parity of the next one; both sides walk the same sequence
-  int seq = 0, stg = 0;
-  uint32_t sph = 0;
-
-  if (warp == CW) {
-    // ================================================================ producer
-    // The row of iteration it: a static stride over the rows, or (dynamic
-    // schedule) the next row of a global counter, taken by rank 0 and sent
-    // to every CTA of the cluster.  Every cluster takes rows until it gets
-    // none, so a launch takes exactly rows + clusters values; the one that
-    // takes the last value resets the counter for the next launch.
-    auto next_row = [&](int it) -> int {
-      if (!p.dyn) {
-        const int r = cid + it * ncl;
-        return r < p.rows ? r : -1;
-      }
-      const int b = it & 1;
-      int r = -1;
-      if (lane == 0) {
-        if (rank == 0) {
-          const unsigned g = atomicAdd(p.grab, 1u);
-          const int rr = g < unsigned(p.rows) ? int(g) : -1;
-          if (g == unsigned(p.rows + ncl - 1)) atomicExch(p.grab, 0u);
-          const uint32_t va = smem_addr(&loc.grab_val[b]), ba = smem_addr(&loc.grab_bar[b]);
-          for (int q = 0; q < S; ++q)
-            st_async_b32(map_rank_addr(va, q), uint32_t(rr), map_rank_addr(ba, q));
-        }
-        mbar_arrive_expect_tx(&loc.grab_bar[b], 4u);
-        wait_cl(&loc.grab_bar[b], uint32_t((it >> 1) & 1));
-        r = loc.grab_val[b];
-      }
-      return __shfl_sync(0xffffffffu, r, 0);
-    };
-    // load the metadata of iteration it's row (or mark the end of the rows)
-    auto issue_meta = [&](int it, int row) {
-      const int b = it & 1;
-      if (it >= 2 && lane == 0) wait_cta(&loc.row_free[b], uint32_t((it >> 1) & 1) ^ 1u);
-      __syncwarp();
-      if (row < 0) {
-        if (lane == 0) {
-          loc.row_id[b] = -1;
-          mbar_arrive(&loc.row_full[b]);
-        }
-        __syncwarp();
-        return;
-      }
-      int nb = N, bad = 0;
-      if (p.seq_budget) {
-        nb = p.seq_budget[row / p.hkv];
-        bad = (nb < 1 || nb > N) ? 1 : 0;
-        nb = min(max(nb, 1), N);
-      }
-      const RowGeo rg = row_geo(nb);
-      const int slot0 = rg.slot0, nvalid = rg.nvalid;
-      int* ps = pos_buf(b);
-      const int32_t* pg = p.pos + size_t(row) * N + slot0;
-      const uint32_t mbytes = uint32_t(G * D * 2 + 2 * D * 2);
-      const bool bulk = p.pos_bulk && (nvalid & 3) == 0;
-      if (!bulk) {
-        for (int j = lane; j < nvalid; j += 32) ps[j] = pg[j];
-        __syncwarp();
-        __threadfence_block();
-      }
-      if (lane == 0) {
-        loc.row_id[b] = row;
-        loc.row_nb[b] = nb;
-        loc.row_bad[b] = bad;
-        const uint32_t pbytes = bulk ? uint32_t(nvalid) * 4 : 0u;
-        mbar_arrive_expect_tx(&loc.row_full[b], mbytes + pbytes);
-        if (pbytes) bulk_copy_g2s(ps, pg, pbytes, &loc.row_full[b]);
-        bulk_copy_g2s(q_buf(b), p.q + size_t(row) * G * D, G * D * 2, &loc.row_full[b]);
-        bulk_copy_g2s(kn_buf(b), p.k_new + size_t(row) * D, D * 2, &loc.row_full[b]);
-        bulk_copy_g2s(vn_buf(b), p.v_new + size_t(row) * D, D * 2, &loc.row_full[b]);
-      }
-      __syncwarp();
-    };
-    auto issue_tiles = [&](int it, int row, int phase) {
-      const int* ps = pos_buf(it & 1);
-      const RowGeo rg = row_geo(loc.row_nb[it & 1]);
-      const int nvalid = rg.nvalid, ntiles = rg.ntiles;
-      const uint16_t* base =
-          (phase == 0 ? p.kcache : p.vcache) + (size_t(row) * N + rg.slot0) * D;
-      for (int tile = 0; tile < ntiles; ++tile) {
-        if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
-        const int s = stg;
-        const uint32_t par = sph;
-        if (lane == 0) {
-          if (seq >= nst) wait_cta(&loc.empty[s], par ^ 1u);
-          const int ns = min(T, nvalid - tile * T);
-          const uint32_t bytes = uint32_t(ns) * D * 2;
-          mbar_arrive_expect_tx(&loc.full[s], bytes);
-          bulk_copy_g2s(ring + size_t(s) * Geo::kTile, base + size_t(tile) * T * D, bytes,
-                        &loc.full[s]);
-        }
-        __syncwarp();
-        ++seq;
-        if (++stg == nst) {
-          stg = 0;
-          sph ^= 1u;
-        }
-      }
-    };
-    int row = next_row(0);
-    issue_meta(0, row);
-    for (int it = 0; row >= 0; ++it) {
-      wait_cta(&loc.row_full[it & 1], uint32_t((it >> 1) & 1));
-      issue_tiles(it, row, 0);
-      const int nrow = next_row(it + 1);
-      issue_meta(it + 1, nrow);
-      issue_tiles(it, row, 1);
-      row = nrow;
-    }
-  } else {
-    // ================================================================ consumers
-    const int sub = lane & 7;   // lane within the slot's 8 lanes (K phase)
-    const int sig = lane >> 3;  // slot within the warp's 4-slot group (K phase)
-    const int perm = GP >= 8 ? sub : GP == 4 ? ((sub >> 1) & 3) : GP == 2 ? ((sub >> 2) & 1) : 0;
-    const int my_head = perm;   // head whose logit this lane holds after the reduction
-    const bool kwriter = ((sub & Geo::BFLY) == 0) && (my_head < G);
-    const int vsub = lane % VL, vslot = lane / VL;
-    // Page-form score only: in V pass u this lane takes the warp's slot pair
-    // u ^ vperm instead of u, so that the per-slot L1 norms of a tile
-    // reduce-scatter over the slot's VL lanes without selects; afterwards
-    // the lane holds the norm of pass vperm's slot.
-    static_assert(VU <= VL && (VU & (VU - 1)) == 0, "norm reduce-scatter");
-    const int vperm = L1V ? (vsub >> (ilog2(VL) - ilog2(VU))) & (VU - 1) : 0;
-    const int eh = lane % GP;   // head of this lane in the probability pass
-    uint32_t xc_uses0 = 0, xc_uses1 = 0;
-
-    for (int it = 0;; ++it) {
-      const int b = it & 1;
-      const uint32_t bpar = uint32_t((it >> 1) & 1);
-      const int* ps = pos_buf(b);
-      wait_cta(&loc.row_full[b], bpar);
-      const int row = loc.row_id[b];
-      if (row < 0) break;
-      const RowGeo rg = row_geo(loc.row_nb[b]);
-      const int slot0 = rg.slot0, nvalid = rg.nvalid, ntiles = rg.ntiles;
-      if (tid == 0 && rank == 0 && loc.row_bad[b]) atomicOr(p.status, LF_STATUS_BAD_SEQ_BUDGET);
-
-      // query heads of the group, fp32, pre-scaled, in this lane's head order
-      float2 qp[GP][DPL / 2];
-      {
-        const uint16_t* qs = q_buf(b);
-#pragma unroll
-        for (int k = 0; k < GP; ++k) {
-          const int h = k ^ perm;
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (h < G) w = *reinterpret_cast<const uint4*>(qs + h * D + c * 64 + sub * 8);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-              qp[k][c * 4 + m] = make_float2(bf16lo(ww[m]) * p.qscale2, bf16hi(ww[m]) * p.qscale2);
-          }
-        }
-      }
-      if (warp == 0) {  // logit of the new token, per head
-        constexpr int DV = D / 32;
-        const uint16_t* qs = q_buf(b);
-        const uint16_t* kn = kn_buf(b);
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-          float a = 0.f;
-#pragma unroll
-          for (int d = 0; d < DV; ++d) {
-            const int dd = lane * DV + d;
-            a = fmaf(__uint_as_float(uint32_t(qs[i * D + dd]) << 16),
-                     __uint_as_float(uint32_t(kn[dd]) << 16), a);
-          }
-#pragma unroll
-          for (int m = 16; m > 0; m >>= 1) a += __shfl_xor_sync(0xffffffffu, a, m);
-          if (lane == 0) loc.s_new[i] = a * p.qscale2;
-        }
-      }
-      {  // newest position and lowest free slot of the chunk
-        int mx = -1, fr = INT_MAX;
-        for (int j = tid; j < nvalid; j += kConsumers) {
-          const int v = ps[j];
-          if (v >= 0) mx = max(mx, v);
-          else fr = min(fr, j);
-        }
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) {
-          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-          fr = min(fr, __shfl_xor_sync(0xffffffffu, fr, m));
-        }
-        if (lane == 0) {
-          loc.wpmax[warp] = mx;
-          loc.wpfree[warp] = fr == INT_MAX ? INT_MAX : slot0 + fr;
-        }
-      }
-      named_barrier(kBarConsumers, kConsumers);
-      bool fastrow = true;  // every slot of the chunk filled: no per-slot masking
-#pragma unroll
-      for (int w = 0; w < CW; ++w) fastrow &= (loc.wpfree[w] == INT_MAX);
-
-      // ---------------------------------------------------------- K phase
-      float rmax = -INFINITY;
-      for (int tile = 0; tile < ntiles; ++tile) {
-        bool tfull = fastrow && (tile + 1) * T <= nvalid;
-        if (!fastrow) {
-          if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
-          tfull = tile_full<T>(ps, tile, nvalid, lane);
-        }
-        wait_cta(&loc.full[stg], sph);
-        const unsigned char* kt = ring + size_t(stg) * Geo::kTile;
-#pragma unroll 1
-        for (int gb = 0; gb < GPW; gb += KU) {
-          float xs[KU];
-#pragma unroll
-          for (int gu = 0; gu < KU; ++gu) {
-            const int si = (warp + (gb + gu) * CW) * 4 + sig;
-            float2 acc[GP];
-#pragma unroll
-            for (int k = 0; k < GP; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-              const uint4 w =
-                  *reinterpret_cast<const uint4*>(kt + si * (2 * D) + c * 128 + sub * 16);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                const float2 kv = make_float2(bf16lo(ww[m]), bf16hi(ww[m]));
-#pragma unroll
-                for (int k = 0; k < GP; ++k) acc[k] = __ffma2_rn(qp[k][c * 4 + m], kv, acc[k]);
-              }
-            }
-            float a[kMaxG];
-#pragma unroll
-            for (int k = 0; k < GP; ++k) a[k] = acc[k].x + acc[k].y;
-            rs_step<GP, 4>(a);
-            rs_step<(GP > 1 ? GP / 2 : 1), 2>(a);
-            rs_step<(GP > 2 ? GP / 4 : 1), 1>(a);
-            xs[gu] = a[0];
-          }
-          if (!tfull) {  // mask free and out-of-range slots
-            const int ns = min(T, nvalid - tile * T);
-#pragma unroll
-            for (int gu = 0; gu < KU; ++gu) {
-              const int si = (warp + (gb + gu) * CW) * 4 + sig;
-              if (!((si < ns) && (ps[tile * T + si] >= 0))) xs[gu] = -INFINITY;
-            }
-          }
-#pragma unroll
-          for (int gu = 0; gu < KU; ++gu) {
-            const int j = tile * T + (warp + (gb + gu) * CW) * 4 + sig;
-            if (kwriter) pl[j * GP + my_head] = xs[gu];
-            rmax = fmaxf(rmax, xs[gu]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&loc.empty[stg]);
-        ++seq;
-        if (++stg == nst) {
-          stg = 0;
-          sph ^= 1u;
-        }
-      }
-      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 8));
-      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 16));
-      if (sig == 0 && kwriter) loc.wmax[warp][my_head] = rmax;
-      named_barrier(kBarConsumers, kConsumers);
-
-      float my_m = -INFINITY;
-      if (G == GP || eh < G) {
-#pragma unroll
-        for (int w = 0; w < CW; ++w) my_m = fmaxf(my_m, loc.wmax[w][eh]);
-      }
-      // 2^(-inf - m) = 0 on the SFU, so masked slots need no select; only a
-      // head with no filled slot in the chunk (m = -inf) needs a finite offset
-      if (my_m == -INFINITY) my_m = 0.f;
-
-      // ---------------------------------------------------------- V phase
-      float2 o[G][4];
-#pragma unroll
-      for (int i = 0; i < G; ++i)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) o[i][m] = make_float2(0.f, 0.f);
-      float lsum = 0.f;
-      float2* ppw = pp + warp * TPW * GP;
-      for (int tile = 0; tile < ntiles; ++tile) {
-        bool tfull = fastrow && (tile + 1) * T <= nvalid;
-        if (!fastrow) {
-          if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
-          tfull = tile_full<T>(ps, tile, nvalid, lane);
-        }
-        wait_cta(&loc.full[stg], sph);
-        const unsigned char* vt = ring + size_t(stg) * Geo::kTile;
-        // probabilities of this warp's slots, kept for the scores and paired for the FMAs
-#pragma unroll
-        for (int idx = lane; idx < TPW * GP; idx += 32) {
-          const int j = tile * T + warp * TPW + idx / GP;
-          float pv = 0.f;
-          if (G == GP || eh < G) {
-            pv = ex2_ftz(pl[j * GP + eh] - my_m);
-            pl[j * GP + eh] = pv;
-          }
-          lsum += pv;
-          ppw[idx] = make_float2(pv, pv);
-        }
-        __syncwarp();
-        const int ns = tfull ? T : min(T, nvalid - tile * T);
-        float pn[kMaxG];  // page-form score: partial L1 norms, by pass
-#pragma unroll VU
-        for (int u = 0; u < TPW / SPV; ++u) {
-          const int ls = (u ^ vperm) * SPV + vslot;
-          const int si = warp * TPW + ls;
-          const uint4 w = *reinterpret_cast<const uint4*>(vt + si * (2 * D) + vsub * 16);
-          float2 v[4] = {make_float2(bf16lo(w.x), bf16hi(w.x)), make_float2(bf16lo(w.y), bf16hi(w.y)),
-                         make_float2(bf16lo(w.z), bf16hi(w.z)), make_float2(bf16lo(w.w), bf16hi(w.w))};
-          if (!tfull) {  // a free or out-of-range slot may hold anything: keep it out
-            const bool valid = (si < ns) && (ps[tile * T + si] >= 0);
-            if (!valid) {
-#pragma unroll
-              for (int m = 0; m < 4; ++m) v[m] = make_float2(0.f, 0.f);
-            }
-          }
-          const float2* pr = ppw + ls * GP;
-          float2 pi[GP];
-          if constexpr (GP >= 2) {
-#pragma unroll
-            for (int h2 = 0; h2 < GP; h2 += 2) {
-              const float4 f = *reinterpret_cast<const float4*>(pr + h2);
-              pi[h2] = make_float2(f.x, f.y);
-              pi[h2 + 1] = make_float2(f.z, f.w);
-            }
-          } else {
-            pi[0] = pr[0];
-          }
-#pragma unroll
-          for (int i = 0; i < G; ++i)
-#pragma unroll
-            for (int m = 0; m < 4; ++m) o[i][m] = __ffma2_rn(pi[i], v[m], o[i][m]);
-          if constexpr (L1V) {
-            float a = 0.f;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) a += fabsf(v[m].x) + fabsf(v[m].y);
-            pn[u] = a;
-          }
-        }
-        if constexpr (L1V) {
-          // the page's score: fold ||v_j||_1 (from the tile already in shared
-          // memory) into the slot's stored probabilities
-          if constexpr (VL == 16) {
-            rs_step<VU, 8>(pn);
-            rs_step<(VU > 1 ? VU / 2 : 1), 4>(pn);
-            rs_step<(VU > 2 ? VU / 4 : 1), 2>(pn);
-            rs_step<(VU > 4 ? VU / 8 : 1), 1>(pn);
-          } else {
-            static_assert(VL == 8, "lanes per slot");
-            rs_step<VU, 4>(pn);
-            rs_step<(VU > 1 ? VU / 2 : 1), 2>(pn);
-            rs_step<(VU > 2 ? VU / 4 : 1), 1>(pn);
-          }
-          constexpr int DUP = VL / VU;  // lanes left holding the same slot's norm
-          const int j = tile * T + warp * TPW + vperm * SPV + vslot;
-          for (int i = vsub & (DUP - 1); i < G; i += DUP) pl[j * GP + i] *= pn[0];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&loc.empty[stg]);
-        ++seq;
-        if (++stg == nst) {
-          stg = 0;
-          sph ^= 1u;
-        }
-      }
-
-      // ---------------------------------------------------- chunk results
-#pragma unroll
-      for (int m = GP; m < 32; m <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
-      if (lane < G) loc.wsum[warp][lane] = lsum;
-#pragma unroll
-      for (int msk = VL; msk < 32; msk <<= 1)
-#pragma unroll
-        for (int i = 0; i < G; ++i)
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            o[i][m].x += __shfl_xor_sync(0xffffffffu, o[i][m].x, msk);
-            o[i][m].y += __shfl_xor_sync(0xffffffffu, o[i][m].y, msk);
-          }
-      if (vslot == 0) {
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-          float4* dst = reinterpret_cast<float4*>(red + (warp * G + i) * D + vsub * 8);
-          dst[0] = make_float4(o[i][0].x, o[i][0].y, o[i][1].x, o[i][1].y);
-          dst[1] = make_float4(o[i][2].x, o[i][2].y, o[i][3].x, o[i][3].y);
-        }
-      }
-      named_barrier(kBarConsumers, kConsumers);
-
-      // ------------------- exchange 1: send this chunk's results to every CTA
-      // (the partial output goes by slices: CTA r combines elements
-      // [r * E / S, (r + 1) * E / S) of the row's output)
-      constexpr int E = G * D;
-      const int per = E / S;  // E is a multiple of 16 and S a power of two <= 16
-      {
-        const uint32_t rxo_l = smem_addr(rxo_buf(b));
-        const uint32_t sc_l = smem_addr(&rx_buf(b)->sc[rank][0]);
-        const uint32_t bar_l = smem_addr(&loc.xa[b]);
-        for (int e4 = tid; e4 < E / 4; e4 += kConsumers) {
-          const int e = e4 * 4;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int w = 0; w < CW; ++w) {
-            const float4 v = *reinterpret_cast<const float4*>(red + w * E + e);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
-          }
-          const int dst = e / per;
-          st_async_v4(map_rank_addr(rxo_l + uint32_t(rank * per + (e - dst * per)) * 4u, dst), acc,
-                      map_rank_addr(bar_l, dst));
-        }
-        if (tid < G) {
-          float mm = -INFINITY, ll = 0.f;
-#pragma unroll
-          for (int w = 0; w < CW; ++w) {
-            mm = fmaxf(mm, loc.wmax[w][tid]);
-            ll += loc.wsum[w][tid];
-          }
-          for (int r = 0; r < S; ++r) {
-            const uint32_t br = map_rank_addr(bar_l, r);
-            st_async_b32(map_rank_addr(sc_l + uint32_t(tid) * 4u, r), __float_as_uint(mm), br);
-            st_async_b32(map_rank_addr(sc_l + uint32_t(GP + tid) * 4u, r), __float_as_uint(ll), br);
-          }
-        }
-        if (tid == 32) {
-          int mx = -1, fr = INT_MAX;
-#pragma unroll
-          for (int w = 0; w < CW; ++w) {
-            mx = max(mx, loc.wpmax[w]);
-            fr = min(fr, loc.wpfree[w]);
-          }
-          const int er = *reinterpret_cast<volatile int*>(&loc.err);
-          for (int r = 0; r < S; ++r) {
-            const uint32_t br = map_rank_addr(bar_l, r);
-            st_async_b32(map_rank_addr(sc_l + uint32_t(2 * GP) * 4u, r), uint32_t(mx), br);
-            st_async_b32(map_rank_addr(sc_l + uint32_t(2 * GP + 1) * 4u, r), uint32_t(fr), br);
-            st_async_b32(map_rank_addr(sc_l + uint32_t(2 * GP + 2) * 4u, r), uint32_t(er), br);
-          }
-        }
-      }
-      // ----------- receive: every CTA's maxima, sums, positions (warp 0 waits)
-      if (warp == 0) {
-        if (lane == 0)
-          mbar_arrive_expect_tx(&loc.xa[b], uint32_t(S) * uint32_t((2 * G + 3) * 4 + per * 4));
-        wait_cl(&loc.xa[b], bpar);
-        // all heads at once: lane = (head i, sender r) with S lanes per head
-        const int HP = 32 / S;  // heads per pass (S is a power of two <= 16)
-        for (int i0 = 0; i0 < G; i0 += HP) {
-          const int i = i0 + lane / S, r = lane % S;
-          const bool ok = i < G;
-          const uint32_t* sc = rx_buf(b)->sc[r];
-          const float m = ok ? __uint_as_float(sc[i]) : -INFINITY;
-          float M = m;
-          for (int o2 = 1; o2 < S; o2 <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
-          const float sn = ok ? loc.s_new[i] : 0.f;
-          M = fmaxf(M, sn);
-          const float cf = ok ? exp2f(m - M) : 0.f;  // 0 for an empty chunk (m = -inf)
-          float lv = ok ? __uint_as_float(sc[GP + i]) * cf : 0.f;
-          for (int o2 = 1; o2 < S; o2 <<= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o2);
-          if (ok) {
-            loc.cf[r][i] = cf;
-            if (r == 0) {
-              loc.Mg[i] = M;
-              loc.Lg[i] = lv + exp2f(sn - M);
-            }
-          }
-        }
-        const bool has = lane < S;
-        const uint32_t* sc = rx_buf(b)->sc[has ? lane : 0];
-        int mx = has ? int(sc[2 * GP]) : -1;
-        int fr = has ? int(sc[2 * GP + 1]) : INT_MAX;
-        int er = has ? int(sc[2 * GP + 2]) : 0;
-        for (int o2 = 1; o2 < S; o2 <<= 1) {
-          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-          fr = min(fr, __shfl_xor_sync(0xffffffffu, fr, o2));
-          er |= __shfl_xor_sync(0xffffffffu, er, o2);
-        }
-        if (lane == 0) {
-          loc.g_t = mx + 1;
-          loc.g_free = fr;
-          loc.g_err = er;
-        }
-      }
-      named_barrier(kBarConsumers, kConsumers);
-      const bool full_row = (loc.g_free == INT_MAX);
-
-      // ------------------------------------------------ scores of own slots
-      if (EVICT) {
-        unsigned long long k1 = kNoKey, k2 = kNoKey;
-        if (full_row && !loc.g_err) {
-          float w[G];
-#pragma unroll
-          for (int i = 0; i < G; ++i) w[i] = loc.cf[rank][i] / loc.Lg[i] * (1.0f / G);
-          const int lim = loc.g_t - p.window;
-          for (int j = tid; j < nvalid; j += kConsumers) {
-            const int gj = slot0 + j;
-            if (gj < p.sink || ps[j] >= lim) continue;
-            float sc = 0.f;
-#pragma unroll
-            for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
-            top2_insert(k1, k2, (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) |
-                                    static_cast<unsigned int>(gj));
-          }
-        }
-        top2_warp(k1, k2);
-        if (lane == 0) {
-          loc.wk1[warp] = k1;
-          loc.wk2[warp] = k2;
-        }
-        named_barrier(kBarConsumers, kConsumers);
-        // ---------------------------- exchange 2: send the keys to every CTA
-        if (warp == 0) {
-          k1 = lane < CW ? loc.wk1[lane] : kNoKey;
-          k2 = lane < CW ? loc.wk2[lane] : kNoKey;
-          top2_warp(k1, k2);
-          if (lane < S) {
-            const uint32_t ka = map_rank_addr(smem_addr(&rx_buf(b)->key[rank][0]), lane);
-            const uint32_t br = map_rank_addr(smem_addr(&loc.xb[b]), lane);
-            st_async_b64(ka, k1, br);
-            st_async_b64(ka + 8u, k2, br);
-          }
-        }
-      }
-
-      // ------------------------------------------ output: this CTA's slice
-      {
-        const int e0 = rank * per;
-        const uint16_t* vn = vn_buf(b);
-        const float* rxo = rxo_buf(b);
-        for (int k = tid; k < per; k += kConsumers) {
-          const int e = e0 + k;
-          const int i = e / D, d = e - i * D;
-          float acc = exp2f(loc.s_new[i] - loc.Mg[i]) * __uint_as_float(uint32_t(vn[d]) << 16);
-          for (int r = 0; r < S; ++r) acc = fmaf(rxo[r * per + k], loc.cf[r][i], acc);
-          p.out[size_t(row) * E + e] = acc / loc.Lg[i];
-        }
-      }
-
-      if (EVICT) {
-        // ----------------------------------- receive: every CTA's keys
-        if (warp == 0) {
-          if (lane == 0) mbar_arrive_expect_tx(&loc.xb[b], uint32_t(S) * 16u);
-          wait_cl(&loc.xb[b], bpar);
-          const bool has = lane < S;
-          unsigned long long g1 = has ? rx_buf(b)->key[lane][0] : kNoKey;
-          unsigned long long g2 = has ? rx_buf(b)->key[lane][1] : kNoKey;
-          top2_warp(g1, g2);
-          if (lane == 0) {
-            int refine = 0;
-            if (g1 != kNoKey && g2 != kNoKey) {
-              const float s1 = __uint_as_float(uint32_t(g1 >> 32));
-              const float s2 = __uint_as_float(uint32_t(g2 >> 32));
-              refine = (s2 <= s1 * (1.0f + kTieRel)) ? 1 : 0;
-            }
-            loc.g_refine = refine;
-            loc.g_slot = (g1 == kNoKey) ? -1 : int(uint32_t(g1 & 0xffffffffull));
-            loc.g_key1 = g1;
-          }
-        }
-        named_barrier(kBarConsumers, kConsumers);
-
-        if (loc.g_refine) {  // the same decision in every CTA of the cluster
-          // fp64 rescoring of the candidates inside the tie band
-          const float s1 = __uint_as_float(uint32_t(loc.g_key1 >> 32));
-          const float thr = s1 * (1.0f + kTieRel);
-          float w[G];
-#pragma unroll
-          for (int i = 0; i < G; ++i) w[i] = loc.cf[rank][i] / loc.Lg[i] * (1.0f / G);
-          const int lim = loc.g_t - p.window;
-          const uint16_t* qs = q_buf(b);
-          double best = INFINITY;
-          int bslot = INT_MAX;
-          // candidates inside the band are found 32 at a time per warp; each is
-          // then rescored by the whole warp (lane l: dims [l*D/32, (l+1)*D/32))
-          constexpr int DL = D / 32;
-          for (int base = warp * 32; base < nvalid; base += kConsumers) {
-            const int j = base + lane;
-            bool in_band = false;
-            if (j < nvalid) {
-              const int gj = slot0 + j;
-              if (gj >= p.sink && ps[j] < lim) {
-                float sc = 0.f;
-#pragma unroll
-                for (int i = 0; i < G; ++i) sc = fmaf(pl[j * GP + i], w[i], sc);
-                in_band = sc <= thr;
-              }
-            }
-            unsigned mask = __ballot_sync(0xffffffffu, in_band);
-            while (mask) {
-              const int src = __ffs(mask) - 1;
-              mask &= mask - 1;
-              const int gj = slot0 + base + src;
-              const uint16_t* krow = p.kcache + (size_t(row) * N + gj) * D + lane * DL;
-              double kv[DL];
-#pragma unroll
-              for (int d = 0; d < DL; ++d) kv[d] = bf16_to_f64(krow[d]);
-              double tot = 0.0;
-#pragma unroll
-              for (int i = 0; i < G; ++i) {
-                double dot = 0.0;
-#pragma unroll
-                for (int d = 0; d < DL; ++d) dot = fma(bf16_to_f64(qs[i * D + lane * DL + d]), kv[d], dot);
-#pragma unroll
-                for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
-                tot += exp2(dot * p.qscale2_64 - double(loc.Mg[i])) / double(loc.Lg[i]);
-              }
-              tot /= double(G);
-              if constexpr (L1V) {
-                const uint16_t* vrow = p.vcache + (size_t(row) * N + gj) * D + lane * DL;
-                double l1 = 0.0;
-#pragma unroll
-                for (int d = 0; d < DL; ++d) l1 += fabs(bf16_to_f64(vrow[d]));
-#pragma unroll
-                for (int m = 16; m > 0; m >>= 1) l1 += __shfl_xor_sync(0xffffffffu, l1, m);
-                tot *= l1;
-              }
-              if (tot < best || (tot == best && gj < bslot)) {
-                best = tot;
-                bslot = gj;
-              }
-            }
-          }
-          if (lane == 0) {
-            loc.wref[warp] = best;
-            loc.wrefs[warp] = bslot;
-          }
-          named_barrier(kBarConsumers, kConsumers);
-          // -------------------- exchange 3: fp64 rescoring results to every CTA
-          const uint32_t xpar = (b ? xc_uses1 : xc_uses0) & 1u;
-          if (b) ++xc_uses1;
-          else ++xc_uses0;
-          if (warp == 0) {
-            double bb = lane < CW ? loc.wref[lane] : INFINITY;
-            int bs = lane < CW ? loc.wrefs[lane] : INT_MAX;
-#pragma unroll
-            for (int m = 16; m > 0; m >>= 1) {
-              const double ob = __shfl_xor_sync(0xffffffffu, bb, m);
-              const int os = __shfl_xor_sync(0xffffffffu, bs, m);
-              if (ob < bb || (ob == bb && os < bs)) {
-                bb = ob;
-                bs = os;
-              }
-            }
-            if (lane < S) {
-              const uint32_t ra = map_rank_addr(smem_addr(&rx_buf(b)->ref[rank][0]), lane);
-              const uint32_t br = map_rank_addr(smem_addr(&loc.xc[b]), lane);
-              st_async_b64(ra, static_cast<unsigned long long>(__double_as_longlong(bb)), br);
-              st_async_b64(ra + 8u, static_cast<unsigned long long>(uint32_t(bs)), br);
-            }
-            if (lane == 0) mbar_arrive_expect_tx(&loc.xc[b], uint32_t(S) * 16u);
-            wait_cl(&loc.xc[b], xpar);
-            const bool has = lane < S;
-            bb = has ? __longlong_as_double(static_cast<long long>(rx_buf(b)->ref[lane][0])) : INFINITY;
-            bs = has ? int(uint32_t(rx_buf(b)->ref[lane][1])) : INT_MAX;
-#pragma unroll
-            for (int m = 16; m > 0; m >>= 1) {
-              const double ob = __shfl_xor_sync(0xffffffffu, bb, m);
-              const int os = __shfl_xor_sync(0xffffffffu, bs, m);
-              if (ob < bb || (ob == bb && os < bs)) {
-                bb = ob;
-                bs = os;
-              }
-            }
-            if (lane == 0 && bs != INT_MAX) loc.g_slot = bs;
-          }
-          named_barrier(kBarConsumers, kConsumers);
-        }
-
-        // -------------------------------------------- in-place eviction
-        if (rank == 0) {
-          int e, ev;
-          if (loc.g_err || loc.err || loc.row_bad[b]) {
-            e = -1;
-            ev = -2;
-          } else if (!full_row) {
-            e = loc.g_free;
-            ev = -1;
-          } else if (loc.g_slot < 0) {
-            e = -1;
-            ev = -2;
-            if (tid == 0) atomicOr(p.status, LF_STATUS_NO_CANDIDATE);
-          } else {
-            e = loc.g_slot;
-            ev = e;
-          }
-          if (e >= 0 && e < N) {
-            constexpr int V16 = D / 8;  // 16-byte vectors per row
-            if (tid < V16) {
-              reinterpret_cast<uint4*>(p.kcache + (size_t(row) * N + e) * D)[tid] =
-                  reinterpret_cast<const uint4*>(kn_buf(b))[tid];
-            } else if (tid < 2 * V16) {
-              reinterpret_cast<uint4*>(p.vcache + (size_t(row) * N + e) * D)[tid - V16] =
-                  reinterpret_cast<const uint4*>(vn_buf(b))[tid - V16];
-            } else if (tid == 2 * V16) {
-              p.pos[size_t(row) * N + e] = loc.g_t;
-            }
-          }
-          if (tid == 0) p.evicted[row] = ev;
-        }
-      }
-      // this row's logits, positions and metadata are no longer needed
-      named_barrier(kBarConsumers, kConsumers);
-      if (tid == 0) mbar_arrive(&loc.row_free[b]);
-    }
-  }
-
-  __syncthreads();
-  // after an error, do not leave with bulk copies still landing in shared memory
-  if (loc.err && tid == kConsumers) {
-    for (int q = max(0, seq - nst); q < seq; ++q)
-      mbar_wait_bounded(&loc.full[q % nst], uint32_t(q / nst) & 1u, kWaitLimitNs);
-  }
-  cluster.sync();  // no CTA leaves while a peer may still read its shared memory
-}
 
 // --------------------------------------------------------------- prefill
 __global__ void prefill_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int n,
@@ -1169,23 +27,49 @@ __global__ void prefill_kernel(const uint4* __restrict__ k, const uint4* __restr
   }
 }
 
+// fp8: quantise the prompt into E4M3 codes (fp32 quotient by the scale,
+// round to nearest even, saturate); one thread per 16 elements
+__global__ void prefill_fp8_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+                                   int n, uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                   int32_t* __restrict__ pos, int budget, int rows, int vec_per_row,
+                                   float k_scale, float v_scale) {
+  const size_t stride = size_t(gridDim.x) * blockDim.x;
+  const size_t tid = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t per_row = size_t(n) * vec_per_row;
+  const size_t total = per_row * rows;
+  for (size_t i = tid; i < total; i += stride) {
+    const size_t r = i / per_row, rest = i - r * per_row;
+    const size_t dst = r * size_t(budget) * vec_per_row + rest;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint16_t* src = (t == 0 ? k : v) + i * 16;
+      const float sc = t == 0 ? k_scale : v_scale;
+      uint32_t w[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(src + 4 * m);
+        const uint32_t c = *reinterpret_cast<const uint32_t*>(src + 4 * m + 2);
+        const uint32_t lo = float2_to_e4m3x2(make_float2(__fdiv_rn(bf16lo(a), sc), __fdiv_rn(bf16hi(a), sc)));
+        const uint32_t hi = float2_to_e4m3x2(make_float2(__fdiv_rn(bf16lo(c), sc), __fdiv_rn(bf16hi(c), sc)));
+        w[m] = (lo & 0xffffu) | (hi << 16);
+      }
+      (t == 0 ? kc : vc)[dst] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  const size_t ptotal = size_t(rows) * budget;
+  for (size_t i = tid; i < ptotal; i += stride) {
+    const int j = int(i % budget);
+    pos[i] = j < n ? j : -1;
+  }
+}
+
 }  // namespace lf
 
 // ======================================================================
 // host side
 // ======================================================================
 
-namespace {
-
-// How one call is laid out on the GPU: S CTAs per row (one cluster), the
-// slots each CTA owns, the ring depth, and how many persistent clusters run.
-struct Plan {
-  int budget;  // the budget the plan was made for (0 = none)
-  int S, chunk, nstages, nclusters;
-  size_t smem;
-};
-
-}  // namespace
+using lf::Plan;
 
 struct lf_ctx {
   int B, Hq, Hkv, D, G, max_budget;
@@ -1198,130 +82,25 @@ struct lf_ctx {
   unsigned int* grab;   // device row counter of the dynamic schedule (after the status word)
   int last_bits;
   int score_mode;  // LF_SCORE_* used by lf_decode_step
-  Plan plan[3];    // [kernel mode]
+  Plan plan[2][3];  // [E4M3 storage][kernel mode]
   unsigned magic;
 };
 
 namespace {
 
 constexpr unsigned kMagic = 0x4c46444bu;
-constexpr int kRowOverheadSlots = 256;  // per-row cost of the exchange, in slot units
 
 bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
 bool valid_handle(lf_handle h) { return h != nullptr && h->magic == kMagic; }
 
-// Slots per CTA: an even split, rounded up to 4 slots (16-byte position rows).
-int chunk_for(int budget, int split) {
-  const int per = (budget + split - 1) / split;
-  return (per + 3) / 4 * 4;
-}
-
-template <int D, int G, int MODE>
-cudaError_t plan_t(const lf_ctx* c, int budget, Plan* out) {
-  using Geo = lf::Geometry<D, G>;
-  auto kern = lf::fused_decode_kernel<D, G, MODE>;
-  static std::mutex mu;
-  static bool attrs_set = false;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!attrs_set) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           c->smem_optin);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-      attrs_set = true;
-    }
-  }
-  const int rows = c->B * c->Hkv;
-  Plan best = {};
-  long long best_cost = -1;
-  const int cands[5] = {1, 2, 4, 8, 16};
-  for (int ci = 0; ci < 5; ++ci) {
-    const int S = cands[ci];
-    if (c->split_override > 0 && S != c->split_override) continue;
-    const int chunk = chunk_for(budget, S);
-    const size_t fixed = Geo::layout(chunk, 0).total;
-    if (fixed + size_t(lf::kMinStages) * Geo::kTile > size_t(c->smem_optin)) continue;
-    int nst = int((size_t(c->smem_optin) - fixed) / Geo::kTile);
-    if (nst > lf::kMaxStages) nst = lf::kMaxStages;
-    const size_t smem = Geo::layout(chunk, nst).total;
-    if (smem > size_t(c->smem_optin)) continue;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(S), unsigned(rows), 1);
-    cfg.blockDim = dim3(Geo::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(S);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int ncl = 0;
-    if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess || ncl < 1) {
-      cudaGetLastError();  // clear a refused size
-      continue;
-    }
-    if (ncl > rows) ncl = rows;
-    const long long iters = (rows + ncl - 1) / ncl;
-    const long long cost = iters * (chunk + kRowOverheadSlots);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best.S = S;
-      best.chunk = chunk;
-      best.nstages = nst;
-      best.nclusters = ncl;
-      best.smem = smem;
-    }
-  }
-  if (best_cost < 0) return cudaErrorInvalidConfiguration;  // no split fits: budget too large
-  best.budget = budget;
-  *out = best;
-  return cudaSuccess;
-}
-
-template <int D, int G, int MODE>
-cudaError_t launch_t(const lf::Params& p, const Plan& pl, cudaStream_t st) {
-  auto kern = lf::fused_decode_kernel<D, G, MODE>;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(pl.S), unsigned(pl.nclusters), 1);
-  cfg.blockDim = dim3(lf::Geometry<D, G>::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = pl.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(pl.S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
-}
-
-#define LF_DISPATCH(D_, G_, CALL)                                                  \
-  do {                                                                             \
-    switch ((D_) * 16 + (G_)) {                                                    \
-      case 64 * 16 + 1: { constexpr int DD = 64, GG = 1; CALL; } break;            \
-      case 64 * 16 + 2: { constexpr int DD = 64, GG = 2; CALL; } break;            \
-      case 64 * 16 + 3: { constexpr int DD = 64, GG = 3; CALL; } break;            \
-      case 64 * 16 + 4: { constexpr int DD = 64, GG = 4; CALL; } break;            \
-      case 64 * 16 + 5: { constexpr int DD = 64, GG = 5; CALL; } break;            \
-      case 64 * 16 + 6: { constexpr int DD = 64, GG = 6; CALL; } break;            \
-      case 64 * 16 + 7: { constexpr int DD = 64, GG = 7; CALL; } break;            \
-      case 64 * 16 + 8: { constexpr int DD = 64, GG = 8; CALL; } break;            \
-      case 128 * 16 + 1: { constexpr int DD = 128, GG = 1; CALL; } break;          \
-      case 128 * 16 + 2: { constexpr int DD = 128, GG = 2; CALL; } break;          \
-      case 128 * 16 + 3: { constexpr int DD = 128, GG = 3; CALL; } break;          \
-      case 128 * 16 + 4: { constexpr int DD = 128, GG = 4; CALL; } break;          \
-      case 128 * 16 + 5: { constexpr int DD = 128, GG = 5; CALL; } break;          \
-      case 128 * 16 + 6: { constexpr int DD = 128, GG = 6; CALL; } break;          \
-      case 128 * 16 + 7: { constexpr int DD = 128, GG = 7; CALL; } break;          \
-      case 128 * 16 + 8: { constexpr int DD = 128, GG = 8; CALL; } break;          \
-      default: break;                                                              \
-    }                                                                              \
-  } while (0)
+// the compiled variants, by [E4M3 storage][kernel mode]
+using PlanFn = cudaError_t (*)(int, int, const lf::PlanIn&, int, Plan*);
+using LaunchFn = cudaError_t (*)(int, int, const lf::Params&, const Plan&, cudaStream_t);
+const PlanFn kPlanFns[2][3] = {{lf::plan_kv2_m0, lf::plan_kv2_m1, lf::plan_kv2_m2},
+                               {lf::plan_kv1_m0, lf::plan_kv1_m1, lf::plan_kv1_m2}};
+const LaunchFn kLaunchFns[2][3] = {{lf::launch_kv2_m0, lf::launch_kv2_m1, lf::launch_kv2_m2},
+                                   {lf::launch_kv1_m0, lf::launch_kv1_m1, lf::launch_kv1_m2}};
 
 // kernel mode of a call: attention only, or eviction by the handle's score
 int kernel_mode(const lf_ctx* c, bool evict) {
@@ -1329,22 +108,15 @@ int kernel_mode(const lf_ctx* c, bool evict) {
   return c->score_mode == LF_SCORE_ALPHA_L1V ? lf::kEvictAlphaL1V : lf::kEvictMeanProb;
 }
 
-cudaError_t get_plan(lf_ctx* c, int budget, int mode, Plan** out) {
-  Plan& pl = c->plan[mode];
+cudaError_t get_plan(lf_ctx* c, int budget, bool fp8, int mode, Plan** out) {
+  Plan& pl = c->plan[fp8 ? 1 : 0][mode];
   if (pl.budget != budget) {
-    cudaError_t e = cudaErrorInvalidValue;
     pl.budget = 0;
-    switch (mode) {
-      case lf::kEvictMeanProb:
-        LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, lf::kEvictMeanProb>(c, budget, &pl)));
-        break;
-      case lf::kEvictAlphaL1V:
-        LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, lf::kEvictAlphaL1V>(c, budget, &pl)));
-        break;
-      default:
-        LF_DISPATCH(c->D, c->G, (e = plan_t<DD, GG, lf::kAttendOnly>(c, budget, &pl)));
-        break;
-    }
+    lf::PlanIn in;
+    in.rows = c->B * c->Hkv;
+    in.split_override = c->split_override;
+    in.smem_optin = c->smem_optin;
+    const cudaError_t e = kPlanFns[fp8 ? 1 : 0][mode](c->D, c->G, in, budget, &pl);
     if (e != cudaSuccess) {
       pl.budget = 0;
       return e;
@@ -1354,11 +126,16 @@ cudaError_t get_plan(lf_ctx* c, int budget, int mode, Plan** out) {
   return cudaSuccess;
 }
 
+bool good_scale(float s) { return s > 0.f && s <= 3.0e38f; }  // positive and finite
+
+// fp8: the cache holds E4M3 codes with scales k_scale / v_scale
 int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
-               uint16_t* kcache, uint16_t* vcache, int32_t* pos, int budget, int sink,
+               void* kcache, void* vcache, int32_t* pos, int budget, int sink,
                int window, float* out, int32_t* evicted, bool evict,
-               const int32_t* seq_budget = nullptr) {
+               const int32_t* seq_budget = nullptr, bool fp8 = false, float k_scale = 1.f,
+               float v_scale = 1.f) {
   if (!valid_handle(h)) return LF_ENOTINIT;
+  if (fp8 && (!good_scale(k_scale) || !good_scale(v_scale))) return LF_EINVAL;
   if (seq_budget && (!aligned(seq_budget, 4) || !h->grab)) return LF_EINVAL;
   if (!q || !k_new || !v_new || !kcache || !vcache || !pos || !out) return LF_EINVAL;
   if (evict && !evicted) return LF_EINVAL;
@@ -1372,7 +149,7 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   const int mode = kernel_mode(h, evict);
   Plan* pl = nullptr;
   {
-    const cudaError_t pe = get_plan(h, budget, mode, &pl);
+    const cudaError_t pe = get_plan(h, budget, fp8, mode, &pl);
     if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
     if (pe != cudaSuccess) return LF_ECUDA;
   }
@@ -1398,21 +175,14 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   p.window = evict ? window : 1;
   p.nstages = pl->nstages;
   p.pos_bulk = (budget % 4 == 0 && aligned(pos, 16)) ? 1 : 0;
-  p.qscale2_64 = 1.4426950408889634 / sqrt(double(h->D));
-  p.qscale2 = float(p.qscale2_64);
+  const double qs2 = 1.4426950408889634 / sqrt(double(h->D));
+  p.qscale2 = float(qs2);
+  p.k_scale = fp8 ? k_scale : 1.f;
+  p.v_scale = fp8 ? v_scale : 1.f;
+  p.qscale2c_64 = qs2 * double(p.k_scale);
+  p.qscale2c = float(p.qscale2c_64);
 
-  cudaError_t e = cudaErrorInvalidValue;
-  switch (mode) {
-    case lf::kEvictMeanProb:
-      LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, lf::kEvictMeanProb>(p, *pl, h->stream)));
-      break;
-    case lf::kEvictAlphaL1V:
-      LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, lf::kEvictAlphaL1V>(p, *pl, h->stream)));
-      break;
-    default:
-      LF_DISPATCH(h->D, h->G, (e = launch_t<DD, GG, lf::kAttendOnly>(p, *pl, h->stream)));
-      break;
-  }
+  const cudaError_t e = kLaunchFns[fp8 ? 1 : 0][mode](h->D, h->G, p, *pl, h->stream);
   return e == cudaSuccess ? LF_OK : LF_ECUDA;
 }
 
@@ -1489,7 +259,8 @@ int lf_set_split(lf_handle h, int split) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (split < 0 || split > lf::kMaxSplit || (split & (split - 1)) != 0) return LF_EINVAL;
   h->split_override = split;
-  for (Plan& pl : h->plan) pl.budget = 0;
+  for (auto& kv : h->plan)
+    for (Plan& pl : kv) pl.budget = 0;
   return LF_OK;
 }
 
@@ -1509,7 +280,7 @@ int lf_get_split(lf_handle h, int budget) {
   if (!valid_handle(h)) return LF_ENOTINIT;
   if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
   Plan* pl = nullptr;
-  const cudaError_t pe = get_plan(h, budget, kernel_mode(h, true), &pl);
+  const cudaError_t pe = get_plan(h, budget, false, kernel_mode(h, true), &pl);
   if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
   if (pe != cudaSuccess) return LF_ECUDA;
   return pl->S;
@@ -1533,6 +304,44 @@ int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, int n, u
       reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), n,
       reinterpret_cast<uint4*>(kcache), reinterpret_cast<uint4*>(vcache), pos, budget, rows, vec);
   return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ECUDA;
+}
+
+int lf_prefill_cache_fp8(lf_handle h, const uint16_t* k, const uint16_t* v, int n, uint8_t* kcache,
+                         uint8_t* vcache, int32_t* pos, int budget, float k_scale, float v_scale) {
+  if (!valid_handle(h)) return LF_ENOTINIT;
+  if (budget < 1 || budget > h->max_budget || n < 0 || n > budget) return LF_EINVAL;
+  if (!good_scale(k_scale) || !good_scale(v_scale)) return LF_EINVAL;
+  if (!kcache || !vcache || !pos || (n > 0 && (!k || !v))) return LF_EINVAL;
+  if (!aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(pos, 4) ||
+      (n > 0 && (!aligned(k, 16) || !aligned(v, 16))))
+    return LF_EINVAL;
+  const int rows = h->B * h->Hkv;
+  const int vec = h->D / 16;  // 16-element groups per row
+  const size_t work = size_t(rows) * (size_t(n) * vec > size_t(budget) ? size_t(n) * vec : size_t(budget));
+  int blocks = int((work + 255) / 256);
+  if (blocks > h->sm_count * 8) blocks = h->sm_count * 8;
+  if (blocks < 1) blocks = 1;
+  lf::prefill_fp8_kernel<<<blocks, 256, 0, h->stream>>>(k, v, n, reinterpret_cast<uint4*>(kcache),
+                                                        reinterpret_cast<uint4*>(vcache), pos, budget,
+                                                        rows, vec, k_scale, v_scale);
+  return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ECUDA;
+}
+
+int lf_decode_step_fp8(lf_handle h, const uint16_t* q, const uint16_t* k_new,
+                       const uint16_t* v_new, uint8_t* kcache, uint8_t* vcache, int32_t* pos,
+                       int budget, const int32_t* seq_budget, int sink, int window,
+                       float k_scale, float v_scale, float* out, int32_t* evicted_idx) {
+  return run_decode(h, q, k_new, v_new, kcache, vcache, pos, budget, sink, window, out,
+                    evicted_idx, true, seq_budget, true, k_scale, v_scale);
+}
+
+int lf_decode_attention_fp8(lf_handle h, const uint16_t* q, const uint16_t* k_new,
+                            const uint16_t* v_new, const uint8_t* kcache, const uint8_t* vcache,
+                            const int32_t* pos, int budget, const int32_t* seq_budget,
+                            float k_scale, float v_scale, float* out) {
+  return run_decode(h, q, k_new, v_new, const_cast<uint8_t*>(kcache),
+                    const_cast<uint8_t*>(vcache), const_cast<int32_t*>(pos), budget, 0, 1, out,
+                    nullptr, false, seq_budget, true, k_scale, v_scale);
 }
 
 int lf_decode_step(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,

@@ -54,6 +54,10 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", default="throughput")
     ap.add_argument("--split", type=int, default=0, help="CTAs per row (0 = automatic)")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="KV cache storage: bf16, or E4M3 codes with one scale per tensor")
+    ap.add_argument("--k-scale", type=float, default=1.0)
+    ap.add_argument("--v-scale", type=float, default=1.0)
     ap.add_argument("--score", default="mean_prob", choices=["mean_prob", "alpha_l1v"],
                     help="eviction score: head-averaged probability (default) or the "
                          "page's attention weight times the value L1 norm")
@@ -70,16 +74,17 @@ def parse():
 
 # ------------------------------------------------------------------ bytes
 
-def algorithmic_bytes(cfg, filled) -> dict:
+def algorithmic_bytes(cfg, filled, kv_bytes: int = 2) -> dict:
     """Bytes one step must move: the K and V of every filled slot once, plus
     every write (fp32 output, the new token's K/V row, its position, the
     evicted index).  q, k_new, v_new and the position table are read too;
     they are listed apart (under 1%).  filled: slots per row, or per
-    sequence ([B], ragged batches)."""
+    sequence ([B], ragged batches).  kv_bytes: bytes per cached element
+    (2 for bf16, 1 for E4M3)."""
     rows = cfg.batch * cfg.hkv
     kv_read = int(np.sum(np.broadcast_to(np.asarray(filled, np.int64), (cfg.batch,)))) \
-        * cfg.hkv * cfg.head_dim * 2 * 2
-    writes = (cfg.batch * cfg.hq * cfg.head_dim * 4 + rows * cfg.head_dim * 2 * 2 + rows * 4
+        * cfg.hkv * cfg.head_dim * kv_bytes * 2
+    writes = (cfg.batch * cfg.hq * cfg.head_dim * 4 + rows * cfg.head_dim * kv_bytes * 2 + rows * 4
               + rows * 4)
     other_reads = (cfg.batch * cfg.hq * cfg.head_dim * 2 + rows * cfg.head_dim * 2 * 2
                    + rows * cfg.budget * 4)
@@ -98,10 +103,13 @@ def measured_peak():
 
 
 def kernel_hash() -> str:
+    """Hash of every kernel source file (the library's csrc directory)."""
     h = hashlib.sha256()
-    for f in (KERNEL_SRC, os.path.join(ROOT, "attention_lf_decode_b200", "csrc", "lf_ptx.cuh")):
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "attention_lf_decode_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as fh:
+                h.update(name.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -170,13 +178,15 @@ class ClockSampler:
 # ------------------------------------------------------------------ oracle
 
 def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_steps: int,
-                score: str = "mean_prob", seq_budget=None):
+                score: str = "mean_prob", seq_budget=None, fp8_scales=None):
     """Time the CPU oracle, as it stands, on sampled batch entries; returns
     (full steps/s extrapolated from rows/s, sample description, steps run)."""
     import oracle
     from attention_lf_decode_b200 import synth
     kc, vc, pos = synth.prefill_layout(kpre_bits[batch_sel], vpre_bits[batch_sel], cfg.budget)
     K, V = synth.bf16_bits_to_f64(kc), synth.bf16_bits_to_f64(vc)
+    if fp8_scales is not None:  # an E4M3 cache: the oracle steps on the codes
+        K, V = oracle.quantize(K, fp8_scales[0]), oracle.quantize(V, fp8_scales[1])
     P = pos.astype(np.int64)
     del kc, vc
     rows = len(batch_sel) * cfg.hkv
@@ -187,8 +197,13 @@ def oracle_rate(cfg, gen, kpre_bits, vpre_bits, seconds: float, batch_sel, max_s
         kn = synth.bf16_bits_to_f64(knb[batch_sel])
         vn = synth.bf16_bits_to_f64(vnb[batch_sel])
         t0 = time.perf_counter()
-        res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window, score=score,
-                                 seq_budget=None if seq_budget is None else seq_budget[batch_sel])
+        nb = None if seq_budget is None else seq_budget[batch_sel]
+        if fp8_scales is None:
+            res = oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window, score=score,
+                                     seq_budget=nb)
+        else:
+            res = oracle.decode_step_fp8(K, V, P, q, kn, vn, cfg.sink, cfg.window, *fp8_scales,
+                                         score=score, seq_budget=nb)
         t_total += time.perf_counter() - t0
         K, V, P = res.kcache, res.vcache, res.pos
         n += 1
@@ -252,11 +267,19 @@ def main():
     binding.lf_set_score(h, score_code)
     split = binding.lf_get_split(h, cfg.budget)
     dev = "cuda"
-    kcache = torch.empty((cfg.batch, cfg.hkv, cfg.budget, cfg.head_dim), dtype=torch.bfloat16, device=dev)
+    fp8 = args.kv == "fp8"
+    kv_bytes = 1 if fp8 else 2
+    kcache = torch.empty((cfg.batch, cfg.hkv, cfg.budget, cfg.head_dim),
+                         dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
     vcache = torch.empty_like(kcache)
     pos = torch.empty((cfg.batch, cfg.hkv, cfg.budget), dtype=torch.int32, device=dev)
-    binding.lf_prefill_cache(h, binding.bf16_from_bits(kpre), binding.bf16_from_bits(vpre),
-                             cfg.prefill, kcache, vcache, pos, cfg.budget)
+    if fp8:
+        binding.lf_prefill_cache_fp8(h, binding.bf16_from_bits(kpre), binding.bf16_from_bits(vpre),
+                                     cfg.prefill, kcache, vcache, pos, cfg.budget,
+                                     args.k_scale, args.v_scale)
+    else:
+        binding.lf_prefill_cache(h, binding.bf16_from_bits(kpre), binding.bf16_from_bits(vpre),
+                                 cfg.prefill, kcache, vcache, pos, cfg.budget)
     q_all = torch.stack([binding.bf16_from_bits(x[0]) for x in inputs])
     kn_all = torch.stack([binding.bf16_from_bits(x[1]) for x in inputs])
     vn_all = torch.stack([binding.bf16_from_bits(x[2]) for x in inputs])
@@ -268,7 +291,10 @@ def main():
     nb_dev = None if nb_host is None else torch.from_numpy(nb_host).to(dev)
 
     def run(q, kn, vn):
-        if nb_dev is None:
+        if fp8:
+            binding.lf_decode_step_fp8(h, q, kn, vn, kcache, vcache, pos, cfg.budget, cfg.sink,
+                                       cfg.window, args.k_scale, args.v_scale, out, ev, nb_dev)
+        elif nb_dev is None:
             binding.lf_decode_step(h, q, kn, vn, kcache, vcache, pos, cfg.budget, cfg.sink,
                                    cfg.window, out, ev)
         else:
@@ -376,7 +402,7 @@ def main():
             raise RuntimeError("device status after e2e")
 
     filled = min(cfg.budget, cfg.prefill) if nb_host is None else np.minimum(nb_host, cfg.prefill)
-    by = algorithmic_bytes(cfg, filled)
+    by = algorithmic_bytes(cfg, filled, kv_bytes)
     kern_s = ms_per_step / 1e3  # one launch per step
     achieved = by["algorithmic"] / kern_s / 1e9
     peak, peak_src = measured_peak()
@@ -385,7 +411,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         rate, sample, _ = oracle_rate(cfg, gen, kpre, vpre, args.cpu_seconds, list(range(4)), 64,
-                                      score=args.score, seq_budget=nb_host)
+                                      score=args.score, seq_budget=nb_host,
+                                      fp8_scales=(args.k_scale, args.v_scale) if fp8 else None)
         cpu = {"value": rate, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
                "sample": sample}
 
@@ -403,7 +430,9 @@ def main():
         "config": {
             "workload": workload, "batch": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv,
             "head_dim": cfg.head_dim, "budget": cfg.budget, "sink": cfg.sink,
-            "window": cfg.window, "kv_dtype": "bf16", "accumulate": "f32",
+            "window": cfg.window,
+            "kv_dtype": (f"e4m3 (k_scale {args.k_scale}, v_scale {args.v_scale})" if fp8 else "bf16"),
+            "accumulate": "f32",
             "parallelism": f"dp{world} (batch per rank, no collective)",
             "split_ctas_per_row": split,
             "seq_budgets": (None if nb_host is None else
@@ -421,7 +450,8 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
                      "bytes_per_launch": by["algorithmic"],
-                     "kernel": f"lf::fused_decode_kernel<{cfg.head_dim},{cfg.group},{1 + score_code}>"},
+                     "kernel": (f"lf::fused_decode_kernel<{cfg.head_dim},{cfg.group},{1 + score_code},"
+                                f"{kv_bytes}>")},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps,
@@ -444,6 +474,16 @@ def reference_arm(args, cfg, workload, world, rank):
     kb, vb = gen.prefill(sel)
     kc, vc, pos = synth.prefill_layout(kb, vb, cfg.budget)
     K, V, P = synth.bf16_bits_to_f64(kc), synth.bf16_bits_to_f64(vc), pos.astype(np.int64)
+    fp8 = args.kv == "fp8"
+    if fp8:  # an E4M3 cache: the oracle steps on the codes
+        K, V = oracle.quantize(K, args.k_scale), oracle.quantize(V, args.v_scale)
+
+    def ostep(K, V, P, q, kn, vn, nb):
+        if fp8:
+            return oracle.decode_step_fp8(K, V, P, q, kn, vn, cfg.sink, cfg.window, args.k_scale,
+                                          args.v_scale, score=args.score, seq_budget=nb)
+        return oracle.decode_step(K, V, P, q, kn, vn, cfg.sink, cfg.window, score=args.score,
+                                  seq_budget=nb)
     budget_s = 150.0
     rows_full = cfg.batch * cfg.hkv
     nb = gen.seq_budgets()  # ragged batch: the sample's budget and every sequence's
@@ -453,9 +493,8 @@ def reference_arm(args, cfg, workload, world, rank):
     # calibrate: one row-step
     qb, knb, vnb = gen.step_inputs(0)
     t0 = time.perf_counter()
-    oracle.decode_step(K[:, :1], V[:, :1], P[:, :1], synth.bf16_bits_to_f64(qb[:1, :cfg.group]),
-                       synth.bf16_bits_to_f64(knb[:1, :1]), synth.bf16_bits_to_f64(vnb[:1, :1]),
-                       cfg.sink, cfg.window, seq_budget=nb0)
+    ostep(K[:, :1], V[:, :1], P[:, :1], synth.bf16_bits_to_f64(qb[:1, :cfg.group]),
+          synth.bf16_bits_to_f64(knb[:1, :1]), synth.bf16_bits_to_f64(vnb[:1, :1]), nb0)
     t_row = time.perf_counter() - t0
     nsteps = args.warmup + args.steps
     rows_per_step = int(max(1, min(cfg.hkv, budget_s / max(nsteps, 1) / max(t_row, 1e-6))))
@@ -467,8 +506,7 @@ def reference_arm(args, cfg, workload, world, rank):
         kn = synth.bf16_bits_to_f64(knb[:1, :heads])
         vn = synth.bf16_bits_to_f64(vnb[:1, :heads])
         t0 = time.perf_counter()
-        res = oracle.decode_step(K[:, :heads], V[:, :heads], P[:, :heads], q, kn, vn,
-                                 cfg.sink, cfg.window, score=args.score, seq_budget=nb0)
+        res = ostep(K[:, :heads], V[:, :heads], P[:, :heads], q, kn, vn, nb0)
         dt = time.perf_counter() - t0
         K[:, :heads], V[:, :heads], P[:, :heads] = res.kcache, res.vcache, res.pos
         if s >= args.warmup:
@@ -484,7 +522,7 @@ def reference_arm(args, cfg, workload, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": workload, "batch": cfg.batch, "budget": cfg.budget,
-                   "score": args.score},
+                   "score": args.score, "kv_dtype": "e4m3" if fp8 else "bf16"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -175,6 +175,44 @@ LF_API int lf_decode_attention_ragged(lf_handle h,
                         const uint16_t* kcache, const uint16_t* vcache, const int32_t* pos,
                         int budget, const int32_t* seq_budget, float* out);
 
+/* FP8 KV storage.  kcache / vcache hold one byte per element: OCP E4M3
+ * codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; S.1111.111 is NaN; largest finite magnitude 448), with one
+ * positive, finite fp32 scale per cache tensor: code c stands for
+ * E4M3(c) * k_scale in kcache and E4M3(c) * v_scale in vcache.  Layouts are
+ * those of the bf16 cache with uint8_t elements: [B, Hkv, budget, D],
+ * 16-byte aligned.  Writing a value x (the prompt in lf_prefill_cache_fp8,
+ * the new token in the step) stores the code of x / scale, the quotient
+ * taken in fp32 (IEEE, correctly rounded) and rounded to the nearest E4M3
+ * value, ties to even; finite quotients beyond +-448 saturate to +-448.
+ * The step is lf_decode_step (or lf_decode_step_ragged when seq_budget is
+ * non-null) on the dequantised cache, decoding in the K and V loops; the
+ * new token takes part in its own step with its exact bf16 k_new / v_new,
+ * and only its stored copy is quantised.  It follows the handle's score.
+ * The pages name 8-bit floats only for another method's medium-importance
+ * tokens (ARKV summary, "Fase de Decodificación": tokens held in low
+ * precision such as FP8 and dequantised on the fly); applying the format to
+ * the whole LongFlow cache is this library's extension.  Returns LF_EINVAL
+ * for a scale that is not positive and finite, or as lf_decode_step. */
+LF_API int lf_prefill_cache_fp8(lf_handle h, const uint16_t* k, const uint16_t* v, int n,
+                         uint8_t* kcache, uint8_t* vcache, int32_t* pos, int budget,
+                         float k_scale, float v_scale);
+
+LF_API int lf_decode_step_fp8(lf_handle h,
+                   const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                   uint8_t* kcache, uint8_t* vcache, int32_t* pos,
+                   int budget, const int32_t* seq_budget, int sink, int window,
+                   float k_scale, float v_scale,
+                   float* out, int32_t* evicted_idx);
+
+/* Attention only over an E4M3 cache (nothing scored or written but out);
+ * seq_budget may be null. */
+LF_API int lf_decode_attention_fp8(lf_handle h,
+                        const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                        const uint8_t* kcache, const uint8_t* vcache, const int32_t* pos,
+                        int budget, const int32_t* seq_budget, float k_scale, float v_scale,
+                        float* out);
+
 /* Eviction score used by later lf_decode_step calls on this handle.
  *   LF_SCORE_MEAN_PROB (default): score_j as documented for lf_decode_step.
  *   LF_SCORE_ALPHA_L1V: the LongFlow summary page's own form (§2B
