@@ -58,6 +58,9 @@ def parse():
                     help="KV cache storage: bf16, or E4M3 codes with one scale per tensor")
     ap.add_argument("--k-scale", type=float, default=1.0)
     ap.add_argument("--v-scale", type=float, default=1.0)
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time the no-eviction control: the same kernel with scoring and "
+                         "eviction compiled out (lf_decode_attention*)")
     ap.add_argument("--score", default="mean_prob", choices=["mean_prob", "alpha_l1v"],
                     help="eviction score: head-averaged probability (default) or the "
                          "page's attention weight times the value L1 norm")
@@ -291,7 +294,16 @@ def main():
     nb_dev = None if nb_host is None else torch.from_numpy(nb_host).to(dev)
 
     def run(q, kn, vn):
-        if fp8:
+        if args.attention_only:
+            if fp8:
+                binding.lf_decode_attention_fp8(h, q, kn, vn, kcache, vcache, pos, cfg.budget,
+                                                args.k_scale, args.v_scale, out, nb_dev)
+            elif nb_dev is None:
+                binding.lf_decode_attention(h, q, kn, vn, kcache, vcache, pos, cfg.budget, out)
+            else:
+                binding.lf_decode_attention_ragged(h, q, kn, vn, kcache, vcache, pos, cfg.budget,
+                                                   nb_dev, out)
+        elif fp8:
             binding.lf_decode_step_fp8(h, q, kn, vn, kcache, vcache, pos, cfg.budget, cfg.sink,
                                        cfg.window, args.k_scale, args.v_scale, out, ev, nb_dev)
         elif nb_dev is None:
@@ -403,6 +415,9 @@ def main():
 
     filled = min(cfg.budget, cfg.prefill) if nb_host is None else np.minimum(nb_host, cfg.prefill)
     by = algorithmic_bytes(cfg, filled, kv_bytes)
+    if args.attention_only:  # the control writes nothing but out
+        by["writes"] = cfg.batch * cfg.hq * cfg.head_dim * 4
+        by["algorithmic"] = by["kv_read"] + by["writes"]
     kern_s = ms_per_step / 1e3  # one launch per step
     achieved = by["algorithmic"] / kern_s / 1e9
     peak, peak_src = measured_peak()
@@ -439,7 +454,9 @@ def main():
                             {"min": int(nb_host.min()), "max": int(nb_host.max()),
                              "mean": float(nb_host.mean()),
                              "schedule": "dynamic (rows taken from a device counter)"}),
-            "score": args.score,
+            "score": None if args.attention_only else args.score,
+            "step": ("attention only (no scoring or eviction)" if args.attention_only
+                     else "fused attention + score + eviction"),
             "l2": "inputs larger than L2: each step reads the 1 GiB K/V cache (L2 is 126 MB)",
             "tokens_per_s": value * cfg.batch,
             "us_per_step_per_layer": ms_per_step * 1e3,
@@ -450,8 +467,8 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
                      "bytes_per_launch": by["algorithmic"],
-                     "kernel": (f"lf::fused_decode_kernel<{cfg.head_dim},{cfg.group},{1 + score_code},"
-                                f"{kv_bytes}>")},
+                     "kernel": (f"lf::fused_decode_kernel<{cfg.head_dim},{cfg.group},"
+                                f"{0 if args.attention_only else 1 + score_code},{kv_bytes}>")},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps,
