@@ -4,6 +4,7 @@
 // translation unit (lf_inst.cu built once per variant) so the variants build
 // in parallel; lf_decode.cu holds the C ABI and dispatches to them.
 #pragma once
+#include <cuda.h>  // CUtensorMap (the type only; no driver library is linked)
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -23,6 +24,9 @@ constexpr int kKvBf16 = 2;
 constexpr int kKvE4m3 = 1;
 
 struct Params {
+  // bf16 storage: the key cache as a 2-D tensor [rows * budget, D] for TMA
+  // tensor copies with 128-byte swizzle (boxes of 64 elements x 128 slots)
+  CUtensorMap kmap;
   const uint16_t* q;      // bf16 [rows * G, D]
   const uint16_t* k_new;  // bf16 [rows, D]
   const uint16_t* v_new;

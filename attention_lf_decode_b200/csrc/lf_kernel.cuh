@@ -95,6 +95,10 @@ struct Local {
   uint64_t xb[2];        // cluster exchange 2 received: candidate keys
   uint64_t xc[2];        // cluster exchange 3 received: fp64 rescoring
   uint64_t grab_bar[2];  // dynamic schedule: the row rank 0 took for this CTA landed
+  uint64_t mma_done[2];  // tensor-core K tile: accumulator [tb] written
+  uint64_t tmem_free[2]; // tensor-core K tile: accumulator [tb] read back
+  uint64_t mma_fin;      // tensor-core: everything issued has completed (exit)
+  uint32_t tmem_base;    // tensor-core: allocated TMEM address
   int grab_val[2];       // dynamic schedule: that row (-1: none left)
   int row_id[2];         // row of a metadata buffer (-1: no more rows)
   int row_nb[2];         // its budget (slots 0 .. nb - 1 exist)
@@ -148,6 +152,23 @@ struct Geometry {
   static constexpr int TPW = T / CW;               // V phase: slots per warp per tile
   static constexpr int VU = TPW / SPV;             // V phase: slot passes per tile
   static constexpr int VUC = VU < VL ? VU : VL;    // V phase: passes per norm reduce-scatter
+  // bf16 storage: Q.K on the tensor cores.  K tiles of TK slots arrive by TMA
+  // tensor copies (KH boxes of 64 elements x TK slots, 128-byte swizzle); one
+  // consumer warp issues tcgen05.mma (M = TK slots, N = 16 heads, K = 16) into
+  // one of two TMEM accumulators; EPI_WG warpgroups read them back, one slot
+  // per thread.
+  static constexpr bool UMMA = KVB == 2;
+  static constexpr int TK = UMMA ? 128 : T;        // slots per K tile
+  static constexpr int KH = D / 64;                // 128-byte halves of a K row
+  static constexpr int KS = D / 16;                // MMAs (k-steps of 16) per K tile
+  static constexpr int kMmaN = 16;
+  static constexpr int kQOpBytes = KH * kMmaN * 128;  // the query heads as the MMA's B operand
+  static constexpr int EPI_WG = CW >= 9 ? 2 : 1;
+  static constexpr int MMA_WARP = CW - 1;
+  static constexpr uint32_t kTmemCols = 32;        // two accumulators of 16 columns
+  static_assert(!UMMA || (TK * ROWB <= kTile && kTile % 1024 == 0 && 4 * EPI_WG <= MMA_WARP &&
+                          GP <= 8 && KH >= 1),
+                "tensor-core K tiles");
   static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
   static constexpr size_t kMetaStride = align128(size_t(G) * D * 2 + 2 * D * 2);
   // per parity: this CTA's slice of every CTA's partial output, then Rx
@@ -159,14 +180,21 @@ struct Geometry {
   struct Layout {
     size_t ring, pl, pos, red, pp, meta, pub, loc, total;
   };
+  __host__ __device__ static size_t align1024(size_t x) { return (x + 1023) & ~size_t(1023); }
+  __host__ __device__ static size_t roundup(size_t x, size_t m) { return (x + m - 1) / m * m; }
   __host__ __device__ static Layout layout(int chunk, int nst) {
     Layout L;
     size_t o = 0;
     L.ring = o; o = align128(o + size_t(nst) * kTile);
     // logits of whole tiles: the last tile of a chunk may be partial
-    L.pl = o;   o = align128(o + size_t((chunk + T - 1) / T * T) * GP * 4);
+    const size_t plslots = roundup(chunk, T) > roundup(chunk, TK) ? roundup(chunk, T) : roundup(chunk, TK);
+    L.pl = o;   o = align128(o + plslots * GP * 4);
     L.pos = o;  o = align128(o + size_t(2) * chunk * 4);
-    L.red = o;  o = align128(o + size_t(CW) * G * D * 4);
+    // the V phase's cross-warp reduction; the K phase's MMA B operand (the
+    // query heads, 1024-byte aligned for the swizzle) shares the space
+    o = UMMA ? align1024(o) : o;
+    const size_t redb = size_t(CW) * G * D * 4;
+    L.red = o;  o = align128(o + (UMMA && size_t(kQOpBytes) > redb ? size_t(kQOpBytes) : redb));
     L.pp = o;   o = align128(o + size_t(CW) * TPW * GP * 8);
     L.meta = o; o = align128(o + 2 * kMetaStride);
     L.pub = o;  o = align128(o + 2 * kPubStride);
@@ -372,7 +400,8 @@ __device__ __forceinline__ void rs_step(float (&a)[NA]) {
 // (evict the lowest head-averaged probability) or kEvictAlphaL1V (evict the
 // lowest head-averaged probability times the L1 norm of the slot's value).
 template <int D, int G, int MODE, int KVB>
-__global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode_kernel(const Params p) {
+__global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
+    fused_decode_kernel(const __grid_constant__ Params p) {
   using Geo = Geometry<D, G, KVB>;
   constexpr bool EVICT = MODE != kAttendOnly;
   constexpr bool L1V = MODE == kEvictAlphaL1V;
@@ -404,7 +433,7 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
     return g;
   };
 
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem[];
   const typename Geo::Layout L = Geo::layout(chunk, nst);
   unsigned char* ring = smem + L.ring;
   float* pl = reinterpret_cast<float*>(smem + L.pl);     // [chunk][GP] logits, then p
@@ -455,11 +484,19 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
       mbar_init(&loc.xb[b], 1);
       mbar_init(&loc.xc[b], 1);
       mbar_init(&loc.grab_bar[b], 1);
+      mbar_init(&loc.mma_done[b], 1);   // the MMA issuer's commit
+      mbar_init(&loc.tmem_free[b], 4);  // the 4 warps of the reading warpgroup
     }
+    mbar_init(&loc.mma_fin, 1);
     loc.err = 0;
     fence_mbar_init();
   }
+  if constexpr (Geo::UMMA) {
+    if (warp == 0) tmem_alloc(&loc.tmem_base, Geo::kTmemCols);
+    tc_fence_before();
+  }
   __syncthreads();
+  if constexpr (Geo::UMMA) tc_fence_after();
   cluster.sync();  // every CTA's barriers exist before the first remote arrival
 
   // ring position: tiles issued (producer) or consumed (consumers) so far, and
@@ -543,6 +580,33 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
       const int* ps = pos_buf(it & 1);
       const RowGeo rg = row_geo(loc.row_nb[it & 1]);
       const int nvalid = rg.nvalid, ntiles = rg.ntiles;
+      if constexpr (Geo::UMMA) {
+        if (phase == 0) {  // K tiles: TMA tensor copies with 128-byte swizzle
+          constexpr int TK = Geo::TK;
+          const int ntk = (nvalid + TK - 1) / TK;
+          const int y0 = row * N + rg.slot0;
+          for (int tile = 0; tile < ntk; ++tile) {
+            if (!tile_filled<TK>(ps, tile, nvalid, lane)) continue;
+            const int s = stg;
+            const uint32_t par = sph;
+            if (lane == 0) {
+              if (seq >= nst) wait_cta(&loc.empty[s], par ^ 1u);
+              mbar_arrive_expect_tx(&loc.full[s], uint32_t(TK * ROWB));
+#pragma unroll
+              for (int h = 0; h < Geo::KH; ++h)
+                tma_load_2d(ring + size_t(s) * Geo::kTile + h * (TK * 128), &p.kmap, h * 64,
+                            y0 + tile * TK, &loc.full[s]);
+            }
+            __syncwarp();
+            ++seq;
+            if (++stg == nst) {
+              stg = 0;
+              sph ^= 1u;
+            }
+          }
+          return;
+        }
+      }
       const unsigned char* base = static_cast<const unsigned char*>(phase == 0 ? p.kcache : p.vcache) +
                                   (size_t(row) * N + rg.slot0) * ROWB;
       for (int tile = 0; tile < ntiles; ++tile) {
@@ -591,6 +655,7 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
     const int vperm = L1V ? (vsub >> (ilog2(VL) - ilog2(VUC))) & (VUC - 1) : 0;
     const int eh = lane % GP;   // head of this lane in the probability pass
     uint32_t xc_uses0 = 0, xc_uses1 = 0;
+    uint32_t kt_count = 0;  // tensor-core K tiles consumed so far (accumulator kt & 1)
 
     for (int it = 0;; ++it) {
       const int b = it & 1;
@@ -604,8 +669,23 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
       if (tid == 0 && rank == 0 && loc.row_bad[b]) atomicOr(p.status, LF_STATUS_BAD_SEQ_BUDGET);
 
       // query heads of the group, fp32, pre-scaled, in this lane's head order
+      // (tensor-core path: the heads as bf16 rows of the MMA's B operand)
       float2 qp[GP][DPL / 2];
-      {
+      if constexpr (Geo::UMMA) {
+        // 16 rows (heads, zero padded) x D, K-major, 128-byte swizzle: 16-byte
+        // chunk c of row r's 128-byte half goes to chunk c ^ (r % 8)
+        const uint16_t* qs = q_buf(b);
+        unsigned char* qop = reinterpret_cast<unsigned char*>(red);
+        for (int i = tid; i < Geo::kMmaN * (D / 8); i += kConsumers) {
+          const int r = i / (D / 8), c8 = i % (D / 8);
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (r < G) w = *reinterpret_cast<const uint4*>(qs + r * D + c8 * 8);
+          const int half = c8 >> 3, c = c8 & 7;
+          *reinterpret_cast<uint4*>(qop + half * (Geo::kMmaN * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                                   ((c ^ (r & 7)) << 4)) = w;
+        }
+        fence_proxy_async_smem();
+      } else {
         const uint16_t* qs = q_buf(b);
 #pragma unroll
         for (int k = 0; k < GP; ++k) {
@@ -667,6 +747,95 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
       for (int w = 0; w < CW; ++w) fastrow &= (loc.wpfree[w] == INT_MAX);
 
       // ---------------------------------------------------------- K phase
+      if constexpr (Geo::UMMA) {
+        // One warp issues the tensor-core MMAs of each K tile into accumulator
+        // kt & 1; a warpgroup reads it back (one slot per thread), frees the
+        // ring stage and the accumulator, and keeps the logits and maxima.
+        constexpr int TK = Geo::TK;
+        constexpr uint32_t idesc = umma_idesc_bf16(TK, Geo::kMmaN);
+        const int ntk = (nvalid + TK - 1) / TK;
+        float hm[GP];
+#pragma unroll
+        for (int k = 0; k < GP; ++k) hm[k] = -INFINITY;
+        const uint32_t qop = smem_addr(red);
+        for (int tile = 0; tile < ntk; ++tile) {
+          if (!fastrow && !tile_filled<TK>(ps, tile, nvalid, lane)) {
+            // a K tile with no filled slot is not loaded; the V phase, whose
+            // tiles are larger, may still read its logits: mask them
+            for (int i = tid; i < TK * GP; i += kConsumers) pl[size_t(tile) * TK * GP + i] = -INFINITY;
+            continue;
+          }
+          const int s = stg;
+          const uint32_t sp = sph;
+          ++seq;
+          if (++stg == nst) {
+            stg = 0;
+            sph ^= 1u;
+          }
+          const int tb = int(kt_count & 1u);
+          const uint32_t up = (kt_count >> 1) & 1u;
+          const int wg = Geo::EPI_WG == 2 ? tb : 0;
+          ++kt_count;
+          if (warp == Geo::MMA_WARP) {
+            if (lane == 0) {
+              wait_cta(&loc.full[s], sp);
+              if (kt_count > 2) wait_cta(&loc.tmem_free[tb], up ^ 1u);
+              tc_fence_after();
+              const uint32_t a0 = smem_addr(ring + size_t(s) * Geo::kTile);
+#pragma unroll
+              for (int kk = 0; kk < Geo::KS; ++kk) {
+                const int h = kk >> 2, k4 = kk & 3;
+                umma_bf16(loc.tmem_base + uint32_t(tb * Geo::kMmaN),
+                          umma_desc_sw128(a0 + h * (TK * 128) + k4 * 32),
+                          umma_desc_sw128(qop + h * (Geo::kMmaN * 128) + k4 * 32), idesc,
+                          kk > 0 ? 1u : 0u);
+              }
+              umma_commit(&loc.mma_done[tb]);
+            }
+            __syncwarp();
+          } else if (warp >> 2 == wg) {
+            wait_cta(&loc.mma_done[tb], up);
+            tc_fence_after();
+            // the tile's keys are consumed: the ring stage may be refilled
+            if ((warp & 3) == 0 && lane == 0) mbar_arrive_count(&loc.empty[s], uint32_t(CW));
+            uint32_t acc[8];
+            tmem_ld8(loc.tmem_base + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(tb * Geo::kMmaN), acc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&loc.tmem_free[tb]);
+            const int j = tile * TK + 32 * (warp & 3) + lane;
+            const bool valid = j < nvalid && (fastrow || ps[j] >= 0);
+            float v[GP];
+#pragma unroll
+            for (int k = 0; k < GP; ++k) {
+              v[k] = valid ? __uint_as_float(acc[k]) * p.qscale2c : -INFINITY;
+              hm[k] = fmaxf(hm[k], v[k]);
+            }
+            if constexpr (GP >= 4) {
+#pragma unroll
+              for (int k = 0; k < GP; k += 4)
+                *reinterpret_cast<float4*>(pl + size_t(j) * GP + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < GP; ++k) pl[size_t(j) * GP + k] = v[k];
+            }
+          }
+        }
+        // the V phase reads whole V tiles: mask the logits past the last K tile
+        {
+          const int end = (nvalid + T - 1) / T * T;
+          for (int i = ntk * TK * GP + tid; i < end * GP; i += kConsumers) pl[i] = -INFINITY;
+        }
+#pragma unroll
+        for (int k = 0; k < GP; ++k) {
+#pragma unroll
+          for (int m = 16; m > 0; m >>= 1) hm[k] = fmaxf(hm[k], __shfl_xor_sync(0xffffffffu, hm[k], m));
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int k = 0; k < GP; ++k) loc.wmax[warp][k] = hm[k];
+        }
+      } else {
       float rmax = -INFINITY;
       for (int tile = 0; tile < ntiles; ++tile) {
         bool tfull = fastrow && (tile + 1) * T <= nvalid;
@@ -730,6 +899,7 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
       rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 8));
       rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 16));
       if (sig == 0 && kwriter) loc.wmax[warp][my_head] = rmax;
+      }
       named_barrier(kBarConsumers, kConsumers);
 
       float my_m = -INFINITY;
@@ -1207,11 +1377,23 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1) fused_decode
     }
   }
 
+  if constexpr (Geo::UMMA) {
+    // every MMA this CTA issued has completed before its TMEM is freed
+    if (warp == Geo::MMA_WARP && lane == 0) {
+      umma_commit(&loc.mma_fin);
+      (void)mbar_wait_bounded(&loc.mma_fin, 0u, kWaitLimitNs);
+    }
+    tc_fence_before();
+  }
   __syncthreads();
   // after an error, do not leave with bulk copies still landing in shared memory
   if (loc.err && tid == kConsumers) {
     for (int q = max(0, seq - nst); q < seq; ++q)
       mbar_wait_bounded(&loc.full[q % nst], uint32_t(q / nst) & 1u, kWaitLimitNs);
+  }
+  if constexpr (Geo::UMMA) {
+    tc_fence_after();
+    if (warp == 0) tmem_free(loc.tmem_base, Geo::kTmemCols);
   }
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }

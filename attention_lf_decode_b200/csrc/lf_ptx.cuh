@@ -1,5 +1,6 @@
-// Thin inline-PTX wrappers for sm_100a: mbarriers, 1-D bulk async copies
-// (global -> shared, completion counted on an mbarrier), the global timer
+// Thin inline-PTX wrappers for sm_100a: mbarriers, 1-D bulk and 2-D tensor
+// (TMA) async copies (global -> shared, completion counted on an mbarrier),
+// tcgen05 tensor-core MMAs with tensor-memory accumulators, the global timer
 // and named barriers.  Written against the public PTX ISA.
 #pragma once
 #include <stdint.h>
@@ -72,6 +73,97 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// mbarrier arrival counting `count` arrivals at once
+__device__ __forceinline__ void mbar_arrive_count(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+// 2-D tiled TMA copy global -> this CTA's shared memory through a tensor map
+// (a __grid_constant__ kernel parameter); completion counted on `bar`.
+// x (the innermost coordinate) times the element size must be a multiple of
+// 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// generic-proxy writes to shared memory -> visible to the async proxy (TMA, tensor cores)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- tcgen05 (5th-generation tensor cores, accumulators in tensor memory)
+// Whole-warp calls: allocate / free `ncols` TMEM columns (a power of two >= 32);
+// the allocated address is written to `slot` in shared memory.
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_addr(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_free(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Shared-memory matrix descriptor: a K-major operand stored in the 128-byte
+// swizzle layout (8-row groups of 128-byte rows, 1024 bytes apart), as a TMA
+// tensor copy with 128-byte swizzle writes it.  `addr` is the byte address of
+// the first 16-element k-block to read (the group base, 1024-byte aligned,
+// plus 32 bytes per k-block of 16 bf16 inside the 128-byte row).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
+  return uint64_t((addr >> 4) & 0x3FFFu)     // start address, 16-byte units
+         | (uint64_t(1) << 16)               // leading byte offset (unused for swizzled K-major)
+         | (uint64_t(1024 >> 4) << 32)       // stride byte offset: next 8-row group
+         | (uint64_t(1) << 46)               // descriptor version (sm_100)
+         | (uint64_t(2) << 61);              // layout: 128-byte swizzle
+}
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, both
+// operands K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+  return (1u << 4)                      // D format: f32
+         | (1u << 7)                    // A format: bf16
+         | (1u << 10)                   // B format: bf16
+         | (uint32_t(N >> 3) << 17)     // N / 8
+         | (uint32_t(M >> 4) << 24);    // M / 16
+}
+// D[tmem] (+)= A[smem] . B[smem]^T, issued by one thread
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on `bar` once every tensor-core operation this thread issued has completed
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+// this warp's 32 TMEM lanes (lane quarter warp % 4), 8 consecutive columns
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // barrier over a subset of the CTA's warps (id 0 is __syncthreads)
