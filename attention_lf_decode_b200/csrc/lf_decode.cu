@@ -129,8 +129,8 @@ cudaError_t get_plan(lf_ctx* c, int budget, bool fp8, int mode, Plan** out) {
 bool good_scale(float s) { return s > 0.f && s <= 3.0e38f; }  // positive and finite
 
 // The key cache as a 2-D tensor [rows * budget, D] of bf16 for TMA tensor
-// copies: boxes of 64 elements x 128 slots, 128-byte swizzle (the layout the
-// tensor-core MMA reads).  The encoder comes from the driver at run time.
+// copies: boxes of 64 elements x (the variant's K tile) slots, 128-byte
+// swizzle (the layout the tensor-core MMA reads).  The encoder comes from the driver at run time.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -148,12 +148,12 @@ EncodeTiledFn encode_fn() {
   });
   return fn;
 }
-int encode_kmap(CUtensorMap* map, const void* kcache, int D, long long slots) {
+int encode_kmap(CUtensorMap* map, const void* kcache, int D, long long slots, int box_slots) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return LF_EUNSUPPORTED;
   const cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(slots)};
   const cuuint64_t strides[1] = {cuuint64_t(D) * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, cuuint32_t(box_slots)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kcache), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -191,7 +191,7 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   lf::Params p;
   memset(&p, 0, sizeof(p));
   if (!fp8) {
-    const int rc = encode_kmap(&p.kmap, kcache, h->D, (long long)h->B * h->Hkv * budget);
+    const int rc = encode_kmap(&p.kmap, kcache, h->D, (long long)h->B * h->Hkv * budget, pl->tk);
     if (rc != LF_OK) return rc;
   }
   p.q = q;

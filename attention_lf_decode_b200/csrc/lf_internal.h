@@ -25,7 +25,7 @@ constexpr int kKvE4m3 = 1;
 
 struct Params {
   // bf16 storage: the key cache as a 2-D tensor [rows * budget, D] for TMA
-  // tensor copies with 128-byte swizzle (boxes of 64 elements x 128 slots)
+  // tensor copies with 128-byte swizzle (boxes of 64 elements x Plan::tk slots)
   CUtensorMap kmap;
   const uint16_t* q;      // bf16 [rows * G, D]
   const uint16_t* k_new;  // bf16 [rows, D]
@@ -58,6 +58,7 @@ struct Params {
 struct Plan {
   int budget;  // the budget the plan was made for (0 = none)
   int S, chunk, nstages, nclusters;
+  int tk;  // slots per K tile (the key tensor map's box height)
   size_t smem;
 };
 

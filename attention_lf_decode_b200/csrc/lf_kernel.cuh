@@ -154,20 +154,25 @@ struct Geometry {
   static constexpr int VUC = VU < VL ? VU : VL;    // V phase: passes per norm reduce-scatter
   // bf16 storage: Q.K on the tensor cores.  K tiles of TK slots arrive by TMA
   // tensor copies (KH boxes of 64 elements x TK slots, 128-byte swizzle); one
-  // consumer warp issues tcgen05.mma (M = TK slots, N = 16 heads, K = 16) into
-  // one of two TMEM accumulators; EPI_WG warpgroups read them back, one slot
-  // per thread.
+  // consumer warp issues tcgen05.mma (NB blocks of M = 128 slots, N = 16
+  // heads, K = 16) into one of two TMEM accumulators; EPI_WG warpgroups read
+  // them back, one slot per thread.
   static constexpr bool UMMA = KVB == 2;
   static constexpr int TK = UMMA ? 128 : T;        // slots per K tile
+  static constexpr int NB = (TK + 127) / 128;      // M = 128 MMA blocks per K tile
+  // both warpgroups read every tile, one block each
+  static constexpr bool EPI_PAIR = CW >= 9 && NB == 2;
   static constexpr int KH = D / 64;                // 128-byte halves of a K row
   static constexpr int KS = D / 16;                // MMAs (k-steps of 16) per K tile
   static constexpr int kMmaN = 16;
   static constexpr int kQOpBytes = KH * kMmaN * 128;  // the query heads as the MMA's B operand
   static constexpr int EPI_WG = CW >= 9 ? 2 : 1;
   static constexpr int MMA_WARP = CW - 1;
-  static constexpr uint32_t kTmemCols = 32;        // two accumulators of 16 columns
+  static constexpr uint32_t kTmemCols = NB == 1 ? 32 : 64;  // two accumulators of NB x 16 columns
+  static constexpr int kReaders = 4 * (EPI_PAIR ? 2 : 1);    // warps reading one accumulator
   static_assert(!UMMA || (TK * ROWB <= kTile && kTile % 1024 == 0 && 4 * EPI_WG <= MMA_WARP &&
-                          GP <= 8 && KH >= 1),
+                          GP <= 8 && KH >= 1 && TK % 8 == 0 && TK <= 256 && NB <= 2 &&
+                          (TK * 128) % 1024 == 0),
                 "tensor-core K tiles");
   static constexpr int BFLY = GP >= 8 ? 0 : GP == 4 ? 1 : GP == 2 ? 3 : 7;
   static constexpr size_t kMetaStride = align128(size_t(G) * D * 2 + 2 * D * 2);
@@ -297,13 +302,15 @@ __device__ __forceinline__ void top2_warp(unsigned long long& k1, unsigned long 
 }
 
 // Any slot of tile `tile` (chunk-local) filled / every slot filled?  Warp-uniform.
+// (T need not be a multiple of 32: every one of the tile's T slots is checked)
 template <int T>
 __device__ __forceinline__ bool tile_filled(const int* ps, int tile, int nvalid, int lane) {
   bool any = false;
 #pragma unroll
-  for (int k = 0; k < T / 32; ++k) {
-    const int j = tile * T + k * 32 + lane;
-    any |= (j < nvalid) && (ps[j] >= 0);
+  for (int k = 0; k < (T + 31) / 32; ++k) {
+    const int o = k * 32 + lane;
+    const int j = tile * T + o;
+    any |= (o < T) && (j < nvalid) && (ps[j] >= 0);
   }
   return __any_sync(0xffffffffu, any);
 }
@@ -311,9 +318,10 @@ template <int T>
 __device__ __forceinline__ bool tile_full(const int* ps, int tile, int nvalid, int lane) {
   bool all = true;
 #pragma unroll
-  for (int k = 0; k < T / 32; ++k) {
-    const int j = tile * T + k * 32 + lane;
-    all &= (j < nvalid) && (ps[j] >= 0);
+  for (int k = 0; k < (T + 31) / 32; ++k) {
+    const int o = k * 32 + lane;
+    const int j = tile * T + o;
+    all &= (o >= T) || ((j < nvalid) && (ps[j] >= 0));
   }
   return __all_sync(0xffffffffu, all);
 }
@@ -485,7 +493,7 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
       mbar_init(&loc.xc[b], 1);
       mbar_init(&loc.grab_bar[b], 1);
       mbar_init(&loc.mma_done[b], 1);   // the MMA issuer's commit
-      mbar_init(&loc.tmem_free[b], 4);  // the 4 warps of the reading warpgroup
+      mbar_init(&loc.tmem_free[b], Geo::kReaders);  // the warps that read an accumulator
     }
     mbar_init(&loc.mma_fin, 1);
     loc.err = 0;
@@ -752,7 +760,8 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
         // kt & 1; a warpgroup reads it back (one slot per thread), frees the
         // ring stage and the accumulator, and keeps the logits and maxima.
         constexpr int TK = Geo::TK;
-        constexpr uint32_t idesc = umma_idesc_bf16(TK, Geo::kMmaN);
+        constexpr uint32_t idesc = umma_idesc_bf16(128, Geo::kMmaN);
+        constexpr int NB = Geo::NB;
         const int ntk = (nvalid + TK - 1) / TK;
         float hm[GP];
 #pragma unroll
@@ -774,8 +783,27 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
           }
           const int tb = int(kt_count & 1u);
           const uint32_t up = (kt_count >> 1) & 1u;
-          const int wg = Geo::EPI_WG == 2 ? tb : 0;
           ++kt_count;
+          const uint32_t tcol = uint32_t(tb * NB * Geo::kMmaN);  // accumulator tb's first column
+          // the warps that read this tile's accumulator, and their blocks
+          bool mine;
+          int bk0, bk1, lead;
+          if constexpr (Geo::EPI_PAIR) {
+            mine = warp < 8;
+            bk0 = warp >> 2;
+            bk1 = bk0 + 1;
+            lead = 0;
+          } else if constexpr (Geo::EPI_WG == 2) {
+            mine = (warp >> 2) == tb;
+            bk0 = 0;
+            bk1 = NB;
+            lead = 4 * tb;
+          } else {
+            mine = warp < 4;
+            bk0 = 0;
+            bk1 = NB;
+            lead = 0;
+          }
           if (warp == Geo::MMA_WARP) {
             if (lane == 0) {
               wait_cta(&loc.full[s], sp);
@@ -783,42 +811,53 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
               tc_fence_after();
               const uint32_t a0 = smem_addr(ring + size_t(s) * Geo::kTile);
 #pragma unroll
-              for (int kk = 0; kk < Geo::KS; ++kk) {
-                const int h = kk >> 2, k4 = kk & 3;
-                umma_bf16(loc.tmem_base + uint32_t(tb * Geo::kMmaN),
-                          umma_desc_sw128(a0 + h * (TK * 128) + k4 * 32),
-                          umma_desc_sw128(qop + h * (Geo::kMmaN * 128) + k4 * 32), idesc,
-                          kk > 0 ? 1u : 0u);
+              for (int bk = 0; bk < NB; ++bk) {
+#pragma unroll
+                for (int kk = 0; kk < Geo::KS; ++kk) {
+                  const int h = kk >> 2, k4 = kk & 3;
+                  umma_bf16(loc.tmem_base + tcol + uint32_t(bk * Geo::kMmaN),
+                            umma_desc_sw128(a0 + h * (TK * 128) + bk * (128 * 128) + k4 * 32),
+                            umma_desc_sw128(qop + h * (Geo::kMmaN * 128) + k4 * 32), idesc,
+                            kk > 0 ? 1u : 0u);
+                }
               }
               umma_commit(&loc.mma_done[tb]);
             }
             __syncwarp();
-          } else if (warp >> 2 == wg) {
+          } else if (mine) {
             wait_cta(&loc.mma_done[tb], up);
             tc_fence_after();
             // the tile's keys are consumed: the ring stage may be refilled
-            if ((warp & 3) == 0 && lane == 0) mbar_arrive_count(&loc.empty[s], uint32_t(CW));
-            uint32_t acc[8];
-            tmem_ld8(loc.tmem_base + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(tb * Geo::kMmaN), acc);
+            if (warp == lead && lane == 0) mbar_arrive_count(&loc.empty[s], uint32_t(CW));
+            for (int bk = bk0; bk < bk1; ++bk) {
+              uint32_t acc[8];
+              tmem_ld8(loc.tmem_base + (uint32_t(32 * (warp & 3)) << 16) + tcol +
+                           uint32_t(bk * Geo::kMmaN),
+                       acc);
+              const int o = bk * 128 + 32 * (warp & 3) + lane;  // slot within the tile
+              if (o < TK) {
+                const int j = tile * TK + o;
+                const bool valid = j < nvalid && (fastrow || ps[j] >= 0);
+                float v[GP];
+#pragma unroll
+                for (int k = 0; k < GP; ++k) {
+                  v[k] = valid ? __uint_as_float(acc[k]) * p.qscale2c : -INFINITY;
+                  hm[k] = fmaxf(hm[k], v[k]);
+                }
+                if constexpr (GP >= 4) {
+#pragma unroll
+                  for (int k = 0; k < GP; k += 4)
+                    *reinterpret_cast<float4*>(pl + size_t(j) * GP + k) =
+                        make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < GP; ++k) pl[size_t(j) * GP + k] = v[k];
+                }
+              }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&loc.tmem_free[tb]);
-            const int j = tile * TK + 32 * (warp & 3) + lane;
-            const bool valid = j < nvalid && (fastrow || ps[j] >= 0);
-            float v[GP];
-#pragma unroll
-            for (int k = 0; k < GP; ++k) {
-              v[k] = valid ? __uint_as_float(acc[k]) * p.qscale2c : -INFINITY;
-              hm[k] = fmaxf(hm[k], v[k]);
-            }
-            if constexpr (GP >= 4) {
-#pragma unroll
-              for (int k = 0; k < GP; k += 4)
-                *reinterpret_cast<float4*>(pl + size_t(j) * GP + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-            } else {
-#pragma unroll
-              for (int k = 0; k < GP; ++k) pl[size_t(j) * GP + k] = v[k];
-            }
           }
         }
         // the V phase reads whole V tiles: mask the logits past the last K tile
@@ -1460,6 +1499,7 @@ cudaError_t plan_t(const PlanIn& c, int budget, Plan* out) {
       best.nstages = nst;
       best.nclusters = ncl;
       best.smem = smem;
+      best.tk = Geo::TK;
     }
   }
   if (best_cost < 0) return cudaErrorInvalidConfiguration;  // no split fits: budget too large

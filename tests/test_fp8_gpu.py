@@ -176,6 +176,16 @@ def test_group_sizes_and_head_dims(Hq, Hkv, D):
     run_steps(c, cfg, kc, vc, pos, 4, rng)
 
 
+def test_appends_across_the_tile_tail():
+    """E4M3 tiles hold 352 slots at D = 128: the filled prefix grows across
+    slots 320..351 of the first tile while the rest stays free."""
+    rng = np.random.default_rng(21)
+    cfg = _custom(2, 8, 2, 128, 700, 4, 8, seed=21)
+    c, kc, vc, pos = _prefilled(cfg, 1.0, 1.0, rng, n=310, split=1)
+    st = run_steps(c, cfg, kc, vc, pos, 50, rng)
+    assert st.appends == 50 * 4
+
+
 def test_appends_then_evicts_and_saturating_values():
     """Prefill 40 of 48 slots; new keys 300x larger than the key scale
     allows, and a value scale of 1/256 (values beyond +-1.75 saturate), so

@@ -123,6 +123,16 @@ def test_budget_covers_length_appends_then_evicts():
     assert st.appends == 8 * 4
 
 
+@pytest.mark.parametrize("D,prefill", [(128, 150), (64, 310)])
+def test_appends_across_every_tile_tail(D, prefill):
+    """One CTA per row, the filled prefix growing one slot per step across the
+    last 32 slots of the first tile (176 slots at D = 128, 352 at D = 64):
+    the free tail of a partly filled tile must stay masked."""
+    cfg = _custom(2, 8, 2, D, 600, 4, 8, seed=D).with_(prefill=prefill)
+    st = H.teacher_forced(cfg, steps=50, split=1)
+    assert st.appends == 50 * 4
+
+
 def test_empty_cache_first_step_returns_v_new():
     cfg = _custom(1, 4, 2, 64, 64, 4, 8, seed=12).with_(prefill=0)
     st = H.teacher_forced(cfg, steps=5)
