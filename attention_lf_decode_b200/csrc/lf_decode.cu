@@ -128,9 +128,9 @@ cudaError_t get_plan(lf_ctx* c, int budget, bool fp8, int mode, Plan** out) {
 
 bool good_scale(float s) { return s > 0.f && s <= 3.0e38f; }  // positive and finite
 
-// The key cache as a 2-D tensor [rows * budget, D] of bf16 for TMA tensor
-// copies: boxes of 64 elements x (the variant's K tile) slots, 128-byte
-// swizzle (the layout the tensor-core MMA reads).  The encoder comes from the driver at run time.
+// A bf16 cache (keys or values) as a 2-D tensor [rows * budget, D] for TMA
+// tensor copies: boxes of 64 elements x (the variant's K or V tile) slots,
+// 128-byte swizzle (the layout the tensor-core MMAs read).  The encoder comes from the driver at run time.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -191,7 +191,9 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   lf::Params p;
   memset(&p, 0, sizeof(p));
   if (!fp8) {
-    const int rc = encode_kmap(&p.kmap, kcache, h->D, (long long)h->B * h->Hkv * budget, pl->tk);
+    const long long slots = (long long)h->B * h->Hkv * budget;
+    int rc = encode_kmap(&p.kmap, kcache, h->D, slots, pl->tk);
+    if (rc == LF_OK && pl->tv > 0) rc = encode_kmap(&p.vmap, vcache, h->D, slots, pl->tv);
     if (rc != LF_OK) return rc;
   }
   p.q = q;

@@ -27,6 +27,7 @@ struct Params {
   // bf16 storage: the key cache as a 2-D tensor [rows * budget, D] for TMA
   // tensor copies with 128-byte swizzle (boxes of 64 elements x Plan::tk slots)
   CUtensorMap kmap;
+  CUtensorMap vmap;  // the value cache likewise (boxes of 64 elements x Plan::tv slots)
   const uint16_t* q;      // bf16 [rows * G, D]
   const uint16_t* k_new;  // bf16 [rows, D]
   const uint16_t* v_new;
@@ -59,6 +60,7 @@ struct Plan {
   int budget;  // the budget the plan was made for (0 = none)
   int S, chunk, nstages, nclusters;
   int tk;  // slots per K tile (the key tensor map's box height)
+  int tv;  // slots per V tile when P.V runs on the tensor cores (the value map's box height), else 0
   size_t smem;
 };
 

@@ -69,6 +69,10 @@ namespace cg = cooperative_groups;
 namespace lf {
 
 constexpr int kMaxCW = 11;                  // most consumer warps of any variant
+// P.V runs on the tensor cores for groups of at least this many (padded) heads
+#ifndef LF_VMMA_MIN_GP
+#define LF_VMMA_MIN_GP 1
+#endif
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 constexpr float kTieRel = 1e-4f;                   // near-tie band rescored in fp64
 constexpr unsigned long long kNoKey = ~0ull;
@@ -98,6 +102,8 @@ struct Local {
   uint64_t mma_done[2];  // tensor-core K tile: accumulator [tb] written
   uint64_t tmem_free[2]; // tensor-core K tile: accumulator [tb] read back
   uint64_t mma_fin;      // tensor-core: everything issued has completed (exit)
+  uint64_t pready[2];    // P.V on the tensor cores: P buffer [pb] written (all consumer warps)
+  uint64_t vdone[2];     // P.V on the tensor cores: the MMAs reading P buffer [pb] completed
   uint32_t tmem_base;    // tensor-core: allocated TMEM address
   int grab_val[2];       // dynamic schedule: that row (-1: none left)
   int row_id[2];         // row of a metadata buffer (-1: no more rows)
@@ -168,7 +174,17 @@ struct Geometry {
   static constexpr int kQOpBytes = KH * kMmaN * 128;  // the query heads as the MMA's B operand
   static constexpr int EPI_WG = CW >= 9 ? 2 : 1;
   static constexpr int MMA_WARP = CW - 1;
-  static constexpr uint32_t kTmemCols = NB == 1 ? 32 : 64;  // two accumulators of NB x 16 columns
+  static constexpr uint32_t kTmemCols = 64;  // two K accumulators (NB x 16 columns each), then O
+  static constexpr uint32_t kOCol = 2 * NB * kMmaN;  // P.V on the tensor cores: O^T's columns
+  // P.V on the tensor cores (bf16, D = 128, not the page-form score): the
+  // V tile is the MN-major A operand (M = 128 dims); the probabilities, split
+  // into bf16 hi + lo parts, are the K-major B operand with N = 32 rows (hi
+  // of the heads in rows 0-15, lo in rows 16-31): [atom of 64 slots][32 rows
+  // x 128 B], double-buffered by V tile.  O^T's hi and lo columns are summed
+  // when read back.
+  static constexpr int NA = (T + 63) / 64;
+  static constexpr int kPBytes = NA * 4096;
+  static constexpr int kMmaNV = 32;
   static constexpr int kReaders = 4 * (EPI_PAIR ? 2 : 1);    // warps reading one accumulator
   static_assert(!UMMA || (TK * ROWB <= kTile && kTile % 1024 == 0 && 4 * EPI_WG <= MMA_WARP &&
                           GP <= 8 && KH >= 1 && TK % 8 == 0 && TK <= 256 && NB <= 2 &&
@@ -187,7 +203,7 @@ struct Geometry {
   };
   __host__ __device__ static size_t align1024(size_t x) { return (x + 1023) & ~size_t(1023); }
   __host__ __device__ static size_t roundup(size_t x, size_t m) { return (x + m - 1) / m * m; }
-  __host__ __device__ static Layout layout(int chunk, int nst) {
+  __host__ __device__ static Layout layout(int chunk, int nst, bool vmma = false) {
     Layout L;
     size_t o = 0;
     L.ring = o; o = align128(o + size_t(nst) * kTile);
@@ -197,10 +213,13 @@ struct Geometry {
     L.pos = o;  o = align128(o + size_t(2) * chunk * 4);
     // the V phase's cross-warp reduction; the K phase's MMA B operand (the
     // query heads, 1024-byte aligned for the swizzle) shares the space
+    // (P.V on the tensor cores: the query operand, then the two P buffers,
+    // instead of the reduction buffer and the probability pairs)
     o = UMMA ? align1024(o) : o;
     const size_t redb = size_t(CW) * G * D * 4;
-    L.red = o;  o = align128(o + (UMMA && size_t(kQOpBytes) > redb ? size_t(kQOpBytes) : redb));
-    L.pp = o;   o = align128(o + size_t(CW) * TPW * GP * 8);
+    const size_t tcb = size_t(kQOpBytes) + (vmma ? 2 * size_t(kPBytes) : 0);
+    L.red = o;  o = align128(o + (vmma ? tcb : (UMMA && tcb > redb ? tcb : redb)));
+    L.pp = o;   o = align128(o + (vmma ? 0 : size_t(CW) * TPW * GP * 8));
     L.meta = o; o = align128(o + 2 * kMetaStride);
     L.pub = o;  o = align128(o + 2 * kPubStride);
     L.loc = o;  o = align128(o + sizeof(Local<GP>));
@@ -413,6 +432,9 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
   using Geo = Geometry<D, G, KVB>;
   constexpr bool EVICT = MODE != kAttendOnly;
   constexpr bool L1V = MODE == kEvictAlphaL1V;
+  // P.V on the tensor cores: bf16, D = 128, and not the page-form score
+  // (which needs |v| of every slot on the CUDA cores)
+  constexpr bool VMMA = Geo::UMMA && !L1V && D == 128 && (Geo::GP >= LF_VMMA_MIN_GP);
   constexpr int CW = Geo::CW, kConsumers = Geo::kConsumers;
   constexpr int T = Geo::T, GP = Geo::GP, DPL = Geo::DPL, ROWB = Geo::ROWB;
   constexpr int NLD = Geo::NLD, LDB = Geo::LDB, EPL = Geo::EPL;
@@ -442,7 +464,7 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
   };
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  const typename Geo::Layout L = Geo::layout(chunk, nst);
+  const typename Geo::Layout L = Geo::layout(chunk, nst, VMMA);
   unsigned char* ring = smem + L.ring;
   float* pl = reinterpret_cast<float*>(smem + L.pl);     // [chunk][GP] logits, then p
   int* pos0 = reinterpret_cast<int*>(smem + L.pos);      // [2][chunk]
@@ -482,7 +504,9 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&loc.full[s], 1);
-      mbar_init(&loc.empty[s], CW);
+      // a stage is released by every consumer warp, or (P.V on the tensor
+      // cores) by the commit of the MMAs that read it
+      mbar_init(&loc.empty[s], VMMA ? 1 : CW);
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
@@ -494,6 +518,8 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
       mbar_init(&loc.grab_bar[b], 1);
       mbar_init(&loc.mma_done[b], 1);   // the MMA issuer's commit
       mbar_init(&loc.tmem_free[b], Geo::kReaders);  // the warps that read an accumulator
+      mbar_init(&loc.pready[b], CW - 1);  // every consumer warp but the MMA issuer
+      mbar_init(&loc.vdone[b], 1);
     }
     mbar_init(&loc.mma_fin, 1);
     loc.err = 0;
@@ -501,6 +527,12 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
   }
   if constexpr (Geo::UMMA) {
     if (warp == 0) tmem_alloc(&loc.tmem_base, Geo::kTmemCols);
+    if constexpr (VMMA) {
+      // the P operands' rows past the group's heads stay zero
+      uint4* pz = reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(red) + Geo::kQOpBytes);
+      for (int i = tid; i < 2 * Geo::kPBytes / 16; i += blockDim.x) pz[i] = make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
+    }
     tc_fence_before();
   }
   __syncthreads();
@@ -614,6 +646,29 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
           }
           return;
         }
+        if constexpr (VMMA) {  // V tiles: TMA tensor copies with 128-byte swizzle
+          const int y0 = row * N + rg.slot0;
+          for (int tile = 0; tile < ntiles; ++tile) {
+            if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
+            const int s = stg;
+            const uint32_t par = sph;
+            if (lane == 0) {
+              if (seq >= nst) wait_cta(&loc.empty[s], par ^ 1u);
+              mbar_arrive_expect_tx(&loc.full[s], uint32_t(T * ROWB));
+#pragma unroll
+              for (int h = 0; h < Geo::KH; ++h)
+                tma_load_2d(ring + size_t(s) * Geo::kTile + h * (T * 128), &p.vmap, h * 64,
+                            y0 + tile * T, &loc.full[s]);
+            }
+            __syncwarp();
+            ++seq;
+            if (++stg == nst) {
+              stg = 0;
+              sph ^= 1u;
+            }
+          }
+          return;
+        }
       }
       const unsigned char* base = static_cast<const unsigned char*>(phase == 0 ? p.kcache : p.vcache) +
                                   (size_t(row) * N + rg.slot0) * ROWB;
@@ -664,6 +719,7 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
     const int eh = lane % GP;   // head of this lane in the probability pass
     uint32_t xc_uses0 = 0, xc_uses1 = 0;
     uint32_t kt_count = 0;  // tensor-core K tiles consumed so far (accumulator kt & 1)
+    uint32_t vt_count = 0;  // tensor-core V tiles consumed so far (P buffer vt & 1)
 
     for (int it = 0;; ++it) {
       const int b = it & 1;
@@ -822,13 +878,16 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
                 }
               }
               umma_commit(&loc.mma_done[tb]);
+              if constexpr (VMMA) umma_commit(&loc.empty[s]);  // the tile's keys are consumed
             }
             __syncwarp();
           } else if (mine) {
             wait_cta(&loc.mma_done[tb], up);
             tc_fence_after();
             // the tile's keys are consumed: the ring stage may be refilled
-            if (warp == lead && lane == 0) mbar_arrive_count(&loc.empty[s], uint32_t(CW));
+            if constexpr (!VMMA) {
+              if (warp == lead && lane == 0) mbar_arrive_count(&loc.empty[s], uint32_t(CW));
+            }
             for (int bk = bk0; bk < bk1; ++bk) {
               uint32_t acc[8];
               tmem_ld8(loc.tmem_base + (uint32_t(32 * (warp & 3)) << 16) + tcol +
@@ -951,12 +1010,111 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
       if (my_m == -INFINITY) my_m = 0.f;
 
       // ---------------------------------------------------------- V phase
+      float lsum = 0.f;
+      float* obuf = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(red) + Geo::kQOpBytes);
+      if constexpr (VMMA) {
+        // P.V on the tensor cores: the consumer threads (all but the MMA
+        // warp) turn their (slot, head) logits into probabilities (kept for
+        // the scores) and write them as bf16 hi + lo into the P operand; the
+        // MMA warp, which only issues, then adds V^T . P^T of the tile to
+        // O^T[dims][heads] in tensor memory.
+        constexpr int kWriters = (CW - 1) * 32;
+        static_assert(kWriters % GP == 0, "head of a writer thread");
+        const bool writer = warp != Geo::MMA_WARP;
+        constexpr uint32_t idesc_v = umma_idesc_bf16(128, Geo::kMmaNV, true);
+        const bool headok = (G == GP || eh < G);
+        unsigned char* Pb = reinterpret_cast<unsigned char*>(obuf);
+        bool any_v = false;
+        for (int tile = 0; tile < ntiles; ++tile) {
+          bool tfull = fastrow && (tile + 1) * T <= nvalid;
+          if (!fastrow) {
+            if (!tile_filled<T>(ps, tile, nvalid, lane)) continue;
+            tfull = tile_full<T>(ps, tile, nvalid, lane);
+          }
+          const int s = stg;
+          const uint32_t sp = sph;
+          ++seq;
+          if (++stg == nst) {
+            stg = 0;
+            sph ^= 1u;
+          }
+          const int pbi = int(vt_count & 1u);
+          const uint32_t vpar = (vt_count >> 1) & 1u;
+          ++vt_count;
+          unsigned char* P = Pb + pbi * Geo::kPBytes;
+          if (writer) {
+          // P buffer pbi was last read by the MMAs of two tiles ago
+          if (vt_count > 2) wait_cta(&loc.vdone[pbi], vpar ^ 1u);
+          for (int idx = tid; idx < T * GP; idx += kWriters) {
+            const int jl = idx / GP;  // idx % GP == eh: kWriters is a multiple of GP
+            const int j = tile * T + jl;
+            float pv = 0.f;
+            if (headok) {
+              pv = ex2_ftz(pl[j * GP + eh] - my_m);
+              pl[j * GP + eh] = pv;
+            }
+            lsum += pv;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(pv - __bfloat162float(hi));
+            // row eh (hi) and 16 + eh (lo) of the slot's 64-slot atom
+            const int off = (jl >> 6) * 4096 + (eh >> 3) * 1024 + (eh & 7) * 128 +
+                            ((((jl & 63) >> 3) ^ (eh & 7)) << 4) + (jl & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(P + off) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(P + off + 2048) = lo;
+          }
+          if (!tfull) {
+            // a free or out-of-range slot's V row may hold anything, NaN
+            // included, and a zero probability does not cancel NaN: zero it
+            wait_cta(&loc.full[s], sp);
+            unsigned char* vt = ring + size_t(s) * Geo::kTile;
+            const int ns = min(T, nvalid - tile * T);
+            for (int idx = tid; idx < T * 16; idx += kWriters) {  // 16-byte chunks of the tile
+              const int jl = idx % T, hc = idx / T;                  // slot, (half, chunk)
+              if (!(jl < ns && ps[tile * T + jl] >= 0))
+                *reinterpret_cast<uint4*>(vt + (hc >> 3) * (T * 128) + jl * 128 + (hc & 7) * 16) =
+                    make_uint4(0, 0, 0, 0);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&loc.pready[pbi]);
+          } else if (lane == 0) {
+            wait_cta(&loc.full[s], sp);
+            wait_cta(&loc.pready[pbi], vpar);
+            tc_fence_after();
+            const uint32_t v0 = smem_addr(ring + size_t(s) * Geo::kTile), p0 = smem_addr(P);
+#pragma unroll 1
+            for (int kk = 0; kk < T / 16; ++kk)
+              umma_bf16(loc.tmem_base + Geo::kOCol, umma_desc_sw128(v0 + kk * 2048, T * 128),
+                        umma_desc_sw128(p0 + (kk >> 2) * 4096 + (kk & 3) * 32), idesc_v,
+                        (any_v || kk > 0) ? 1u : 0u);
+            umma_commit(&loc.vdone[pbi]);
+            umma_commit(&loc.empty[s]);  // the tile's values are consumed
+          }
+          __syncwarp();
+          any_v = true;
+        }
+        // the row's partial output: O^T from tensor memory (one dim per thread)
+        if (any_v) {
+          wait_cta(&loc.vdone[(vt_count - 1) & 1u], ((vt_count - 1) >> 1) & 1u);
+          tc_fence_after();
+        }
+        if (warp < 4) {
+          uint32_t rh[8], rl[8];  // the hi and lo halves of O^T for this dim
+          tmem_ld8(loc.tmem_base + (uint32_t(32 * warp) << 16) + Geo::kOCol, rh);
+          tmem_ld8(loc.tmem_base + (uint32_t(32 * warp) << 16) + Geo::kOCol + 16, rl);
+          const int d = 32 * warp + lane;
+#pragma unroll
+          for (int i = 0; i < G; ++i)
+            obuf[i * D + d] = any_v ? __uint_as_float(rh[i]) + __uint_as_float(rl[i]) : 0.f;
+          tc_fence_before();
+        }
+      } else {
       float2 o[G][4];
 #pragma unroll
       for (int i = 0; i < G; ++i)
 #pragma unroll
         for (int m = 0; m < 4; ++m) o[i][m] = make_float2(0.f, 0.f);
-      float lsum = 0.f;
       float2* ppw = pp + warp * TPW * GP;
       for (int tile = 0; tile < ntiles; ++tile) {
         bool tfull = fastrow && (tile + 1) * T <= nvalid;
@@ -1047,10 +1205,6 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
         }
       }
 
-      // ---------------------------------------------------- chunk results
-#pragma unroll
-      for (int m = GP; m < 32; m <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
-      if (lane < G) loc.wsum[warp][lane] = lsum;
 #pragma unroll
       for (int msk = VL; msk < 32; msk <<= 1)
 #pragma unroll
@@ -1068,6 +1222,11 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
           dst[1] = make_float4(o[i][2].x, o[i][2].y, o[i][3].x, o[i][3].y);
         }
       }
+      }
+      // ---------------------------------------------------- chunk results
+#pragma unroll
+      for (int m = GP; m < 32; m <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
+      if (lane < G) loc.wsum[warp][lane] = lsum;
       named_barrier(kBarConsumers, kConsumers);
 
       // ------------------- exchange 1: send this chunk's results to every CTA
@@ -1082,13 +1241,17 @@ __global__ void __launch_bounds__(Geometry<D, G, KVB>::kThreads, 1)
         for (int e4 = tid; e4 < E / 4; e4 += kConsumers) {
           const int e = e4 * 4;
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          if constexpr (VMMA) {
+            acc = *reinterpret_cast<const float4*>(obuf + e);
+          } else {
 #pragma unroll
-          for (int w = 0; w < CW; ++w) {
-            const float4 v = *reinterpret_cast<const float4*>(red + w * E + e);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+            for (int w = 0; w < CW; ++w) {
+              const float4 v = *reinterpret_cast<const float4*>(red + w * E + e);
+              acc.x += v.x;
+              acc.y += v.y;
+              acc.z += v.z;
+              acc.w += v.w;
+            }
           }
           if constexpr (KVB == 1) {  // E4M3 values were summed without their scale
             acc.x *= p.v_scale;
@@ -1467,11 +1630,13 @@ cudaError_t plan_t(const PlanIn& c, int budget, Plan* out) {
     const int S = cands[ci];
     if (c.split_override > 0 && S != c.split_override) continue;
     const int chunk = chunk_for(budget, S);
-    const size_t fixed = Geo::layout(chunk, 0).total;
+    constexpr bool vmma = KVB == 2 && MODE != kEvictAlphaL1V && D == 128 &&
+                          (Geo::GP >= LF_VMMA_MIN_GP);
+    const size_t fixed = Geo::layout(chunk, 0, vmma).total;
     if (fixed + size_t(kMinStages) * Geo::kTile > size_t(c.smem_optin)) continue;
     int nst = int((size_t(c.smem_optin) - fixed) / Geo::kTile);
     if (nst > kMaxStages) nst = kMaxStages;
-    const size_t smem = Geo::layout(chunk, nst).total;
+    const size_t smem = Geo::layout(chunk, nst, vmma).total;
     if (smem > size_t(c.smem_optin)) continue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(S), unsigned(rows), 1);
@@ -1500,6 +1665,7 @@ cudaError_t plan_t(const PlanIn& c, int budget, Plan* out) {
       best.nclusters = ncl;
       best.smem = smem;
       best.tk = Geo::TK;
+      best.tv = vmma ? Geo::T : 0;
     }
   }
   if (best_cost < 0) return cudaErrorInvalidConfiguration;  // no split fits: budget too large

@@ -124,19 +124,23 @@ __device__ __forceinline__ void tc_fence_after() {
 // tensor copy with 128-byte swizzle writes it.  `addr` is the byte address of
 // the first 16-element k-block to read (the group base, 1024-byte aligned,
 // plus 32 bytes per k-block of 16 bf16 inside the 128-byte row).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
+// For an MN-major operand (the MN dimension contiguous in the 128-byte rows,
+// 8 K-rows per 1024-byte atom) `lbo` is the byte stride between 64-element
+// MN atoms.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr, uint32_t lbo = 16) {
   return uint64_t((addr >> 4) & 0x3FFFu)     // start address, 16-byte units
-         | (uint64_t(1) << 16)               // leading byte offset (unused for swizzled K-major)
+         | (uint64_t((lbo >> 4) & 0x3FFFu) << 16)  // leading byte offset (K-major: unused)
          | (uint64_t(1024 >> 4) << 32)       // stride byte offset: next 8-row group
          | (uint64_t(1) << 46)               // descriptor version (sm_100)
          | (uint64_t(2) << 61);              // layout: 128-byte swizzle
 }
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, both
-// operands K-major, M x N.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, B
+// K-major, A K-major or MN-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major = false) {
   return (1u << 4)                      // D format: f32
          | (1u << 7)                    // A format: bf16
          | (1u << 10)                   // B format: bf16
+         | (a_mn_major ? (1u << 15) : 0u)  // A major-ness: 0 = K-major, 1 = MN-major
          | (uint32_t(N >> 3) << 17)     // N / 8
          | (uint32_t(M >> 4) << 24);    // M / 16
 }
