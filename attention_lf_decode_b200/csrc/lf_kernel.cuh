@@ -12,39 +12,43 @@
 // into on-chip memory).
 //
 // Design.  One row = one (batch, KV head) pair; its K and V slabs are each
-// [budget, D] bf16, contiguous.
+// [budget, D] of bf16 or E4M3 codes, contiguous.
 //   * Persistent thread-block clusters: a cluster of S CTAs owns a row at a
-//     time and splits its slots into S chunks (flash-decoding split); the
-//     cluster then moves on to row + (number of clusters).  Each CTA has 8
-//     consumer warps and 1 producer warp.
-//   * The producer streams the chunk's K tiles, then its V tiles (16 KB each,
-//     contiguous) with 1-D bulk async copies into an mbarrier-guarded ring,
-//     without a pause between rows: while the consumers finish one row, the
-//     next row's position table, query heads and new K/V are already loaded
-//     and its first tiles are in flight.  Tiles whose slots are all free are
-//     never loaded.  No multicast: every CTA fetches its own tiles.
-//   * K phase: 8 lanes per slot, 16-byte conflict-free shared loads, packed
-//     fp32x2 FMAs against the pre-scaled query heads held in registers in a
-//     per-lane head order that lets the 8-lane reduce-scatter run without
-//     selects.  Logits (log2 domain) stay in shared memory: the exact
-//     normalised probabilities need the row-wide max and sum, which only
-//     exist once every CTA of the cluster is done.
-//   * V phase: p = 2^(s - m_cta) in place, o += p * v with 8 dims per lane
-//     and packed FMAs.
-//   * Cluster exchange through distributed shared memory, signalled by
-//     remote mbarrier arrivals (release / acquire at cluster scope) into
-//     per-row-parity buffers, so no whole-cluster barrier stops the
-//     producer: row max / sum per head, newest position, lowest free slot;
-//     then each CTA scores its own slots (exact normalised probability
-//     averaged over the group's heads), reduces packed (fp32 score bits << 32
-//     | slot) keys to the two lowest, and combines its share of the output.
+//     time and splits its slots evenly (flash-decoding split); rows come from
+//     a static stride, or (ragged batches) from a device counter that rank 0
+//     reads and pushes to its peers.  A CTA has 11 consumer warps (8 for
+//     groups of more than 4 heads) and 1 producer warp.
+//   * The producer streams the chunk's K tiles, then its V tiles, into an
+//     mbarrier-guarded ring without a pause between rows: while the
+//     consumers finish one row, the next row's position table, query heads
+//     and new K/V are loaded and its first tiles are in flight.  Tiles whose
+//     slots are all free are never loaded.  No multicast.
+//   * K phase, bf16: 128-slot K tiles by TMA tensor copies with 128-byte
+//     swizzle; one consumer warp issues tcgen05.mma (M = 128 slots, N = 16
+//     heads, K = 16) into a double-buffered TMEM accumulator; a warpgroup
+//     reads it back with tcgen05.ld, one slot per thread.  E4M3: 1-D bulk
+//     tiles, 8 lanes per slot, packed fp32x2 FMAs against pre-scaled query
+//     heads held in a per-lane head order that lets the 8-lane reduce-scatter
+//     run without selects.  Logits (log2 domain) stay in shared memory: the
+//     exact normalised probabilities need the row-wide max and sum, which
+//     only exist once every CTA of the cluster is done.
+//   * V phase: p = 2^(s - m_cta), kept for the scores.  8-head groups with
+//     bf16 at D = 128: TMA-swizzled V tiles, P as bf16 hi + lo rows of an
+//     N = 32 tcgen05 B operand, O^T accumulated in TMEM.  Otherwise: o += p v
+//     with 8 elements per lane and packed FMAs (the page-form score also sums
+//     |v| there).
+//   * Cluster exchange through distributed shared memory by st.async pushes
+//     into per-row-parity buffers, completing bytes on the receiver's
+//     mbarrier: row max / sum per head, newest position, lowest free slot and
+//     the partial outputs; then each CTA scores its own slots (exact
+//     normalised probability averaged over the group's heads, optionally
+//     times ||v||_1), reduces packed (fp32 score bits << 32 | slot) keys to
+//     the two lowest, and combines its share of the output.
 //   * Near ties (two lowest scores within a relative 1e-4) are rescored in
 //     fp64 from the cache, so the choice follows the exact ranking.
-//   * KV storage is bf16 or E4M3 (one byte per element, one scale per cache
-//     tensor, decoded in the K and V loops; the new token is written
-//     quantised with round-to-nearest-even and saturation).
-//   * CTA rank 0 writes k_new / v_new / t into the chosen slot after the key
-//     exchange, which every CTA enters only after its last read of the row.
+//   * CTA rank 0 writes k_new / v_new / t into the chosen slot (E4M3: the
+//     quantised codes) after the key exchange, which every CTA enters only
+//     after its last read of the row.
 #pragma once
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
