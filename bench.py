@@ -293,7 +293,7 @@ def main():
     nb_host = gen.seq_budgets()
     nb_dev = None if nb_host is None else torch.from_numpy(nb_host).to(dev)
 
-    def run(q, kn, vn):
+    def run(q, kn, vn, out=out, ev=ev):
         if args.attention_only:
             if fp8:
                 binding.lf_decode_attention_fp8(h, q, kn, vn, kcache, vcache, pos, cfg.budget,
@@ -366,50 +366,83 @@ def main():
     ms_per_step = ms_max / args.steps
     value = scaling.whole_job_rate(world, args.steps, ms_max)
 
-    # end to end: pinned host inputs -> device, step, result -> pinned host, every step
+    # End to end, through the public call: every step copies its inputs from
+    # pinned host memory to the device, runs lf_decode_step, copies out and
+    # evicted_idx back to pinned host memory, and the host reads that result.
+    # The steps are pipelined two deep: copies run on a second stream into
+    # double-buffered device and host buffers, so step i's copies overlap
+    # steps i - 1 and i + 1, and the host reads step i's result once step
+    # i + 2 has been enqueued.
     e2e = None
     if not args.no_e2e:
         hq = torch.from_numpy(np.stack([x[0] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
         hk = torch.from_numpy(np.stack([x[1] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
         hv = torch.from_numpy(np.stack([x[2] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
-        d_q = torch.empty_like(q_all[0])
-        d_k = torch.empty_like(kn_all[0])
-        d_v = torch.empty_like(vn_all[0])
-        h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-        h_ev = torch.empty(ev.shape, dtype=torch.int32).pin_memory()
+        NBUF = 2
+        cs = torch.cuda.Stream()
+        d_in = [(torch.empty_like(q_all[0]), torch.empty_like(kn_all[0]), torch.empty_like(vn_all[0]))
+                for _ in range(NBUF)]
+        d_out = [out] + [torch.empty_like(out) for _ in range(NBUF - 1)]
+        d_ev = [ev] + [torch.empty_like(ev) for _ in range(NBUF - 1)]
+        h_out = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(NBUF)]
+        h_ev = [torch.empty(ev.shape, dtype=torch.int32).pin_memory() for _ in range(NBUF)]
+        ev_h2d = [torch.cuda.Event() for _ in range(NBUF)]
+        ev_k = [torch.cuda.Event() for _ in range(NBUF)]
+        ev_d2h = [torch.cuda.Event() for _ in range(NBUF)]
+        pending = []  # buffers whose step's result the host has not read yet
+        results = []
         n_e2e = args.e2e_steps
 
+        def consume():
+            b = pending.pop(0)
+            ev_d2h[b].synchronize()
+            results.append(float(h_out[b][0, 0, 0]))  # the host reads the step's result
+
         def e2e_step(i):
+            b = i % NBUF
             j = i % n_inputs
-            d_q.copy_(hq[j], non_blocking=True)
-            d_k.copy_(hk[j], non_blocking=True)
-            d_v.copy_(hv[j], non_blocking=True)
-            run(d_q, d_k, d_v)
-            h_out.copy_(out, non_blocking=True)
-            h_ev.copy_(ev, non_blocking=True)
-            stream.synchronize()
-            return float(h_out[0, 0, 0])  # the host reads the step's result
+            if len(pending) == NBUF:  # buffer b is free once its last step's result is read
+                consume()
+            with torch.cuda.stream(cs):
+                for dst, src in zip(d_in[b], (hq[j], hk[j], hv[j])):
+                    dst.copy_(src, non_blocking=True)
+                ev_h2d[b].record(cs)
+            stream.wait_event(ev_h2d[b])
+            run(*d_in[b], out=d_out[b], ev=d_ev[b])
+            ev_k[b].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_k[b])
+                h_out[b].copy_(d_out[b], non_blocking=True)
+                h_ev[b].copy_(d_ev[b], non_blocking=True)
+                ev_d2h[b].record(cs)
+            pending.append(b)
 
         for i in range(3):
             e2e_step(i)
+        while pending:
+            consume()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
+        a0.record(cs)
         for i in range(n_e2e):
             e2e_step(i)
-        a1.record(stream)
+        a1.record(cs)
+        while pending:
+            consume()
         a1.synchronize()
         ems = scaling.max_over_ranks(a0.elapsed_time(a1), dev)
-        h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
-        d2h = h_out.numel() * 4 + h_ev.numel() * 4
+        h2d = sum(t.numel() for t in d_in[0]) * 2
+        d2h = h_out[0].numel() * 4 + h_ev[0].numel() * 4
         e2e = {"value": scaling.whole_job_rate(world, n_e2e, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": ems / n_e2e,
                "note": "per step: pinned H2D of q/k_new/v_new, lf_decode_step, D2H of out and "
-                       "evicted_idx, stream sync; the KV cache stays resident"}
+                       "evicted_idx, host read of the result; pipelined two steps deep on a "
+                       "copy stream with double-buffered inputs and outputs; the KV cache "
+                       "stays resident"}
         if binding.lf_get_status(h) != binding.LF_OK:
             raise RuntimeError("device status after e2e")
 
