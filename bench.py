@@ -38,7 +38,6 @@ sys.path.insert(0, ROOT)
 METRIC = "fused decode steps/s per layer and achieved HBM GB/s vs B200 peak"
 UNIT = "steps/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "attention_lf_decode_b200", "csrc", "lf_decode.cu")
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_decode_throughput_b64_n4096.md")
 
 
