@@ -120,8 +120,10 @@ LF_API int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, i
  * LF_STATUS_NO_CANDIDATE, writes evicted = -2 and leaves the row's cache
  * unchanged when a full row has no candidate.
  * A budget too large for one thread-block cluster of at most 16 CTAs to
- * hold the row's logits in shared memory (about 32K slots at G = 4,
- * D = 128; less for larger G) is rejected with LF_EINVAL.
+ * hold the row's logits in shared memory is rejected with LF_EINVAL, before
+ * anything is enqueued.  Measured on a B200: budgets up to 65,536 slots plan
+ * for groups of up to 4 heads (98,304 do not), and up to 49,152 for 5 to 8
+ * heads (65,536 do not); lf_get_split answers the question for a budget.
  * Near ties: scores are computed in fp32; when the two lowest candidate
  * scores of a row are within a relative 1e-4 of each other, the kernel
  * rescores those candidates in fp64 before choosing. */

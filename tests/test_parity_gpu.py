@@ -133,6 +133,19 @@ def test_appends_across_every_tile_tail(D, prefill):
     assert st.appends == 50 * 4
 
 
+def test_budget_beyond_shared_memory_is_rejected_on_the_host():
+    """A budget whose per-CTA logits cannot fit in shared memory even at
+    16 CTAs per row is rejected with LF_EINVAL before anything is launched;
+    a large feasible budget gets a split."""
+    h = binding.lf_init(1, 8, 2, 128, 1 << 21)
+    try:
+        lib = binding.load_library()
+        assert lib.lf_get_split(h.ptr, 1 << 21) == binding.LF_EINVAL
+        assert lib.lf_get_split(h.ptr, 16384) in (1, 2, 4, 8, 16)
+    finally:
+        binding.lf_destroy(h)
+
+
 def test_empty_cache_first_step_returns_v_new():
     cfg = _custom(1, 4, 2, 64, 64, 4, 8, seed=12).with_(prefill=0)
     st = H.teacher_forced(cfg, steps=5)
