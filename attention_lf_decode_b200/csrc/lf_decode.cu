@@ -192,6 +192,7 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
   memset(&p, 0, sizeof(p));
   if (!fp8) {
     const long long slots = (long long)h->B * h->Hkv * budget;
+    if (slots >= (1LL << 31)) return LF_EINVAL;  // TMA slot coordinates are 32-bit
     int rc = encode_kmap(&p.kmap, kcache, h->D, slots, pl->tk);
     if (rc == LF_OK && pl->tv > 0) rc = encode_kmap(&p.vmap, vcache, h->D, slots, pl->tv);
     if (rc != LF_OK) return rc;
