@@ -69,8 +69,11 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay a captured CUDA graph of the timed steps; its kernel nodes "
+                         "hold fixed inputs, so new tokens repeat every graph length")
     ap.add_argument("--no-graph", action="store_true",
-                    help="launch every step from Python instead of replaying a captured CUDA graph")
+                    help="launch every step from Python (the default)")
     return ap.parse_args()
 
 
@@ -312,9 +315,35 @@ def main():
             binding.lf_decode_step_ragged(h, q, kn, vn, kcache, vcache, pos, cfg.budget, nb_dev,
                                           cfg.sink, cfg.window, out, ev)
 
+    # Every step's new token is distinct: re-inserting a token already cached
+    # would tie its score exactly with its copy's and send that row through
+    # the fp64 rescoring, which real decoding does not do.  The new K/V of the
+    # steps are drawn on the device with the synthetic recipe (N(0, 1); key
+    # outliers along u when the config has them); the queries cycle through
+    # the seeded sets.
+    u_dev = torch.from_numpy(gen.u).to(dev)
+
+    def draw_new_kv(n, seed):
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        shape = (n, cfg.batch, cfg.hkv, cfg.head_dim)
+        kn = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        vn = torch.empty_like(kn)
+        for c0 in range(0, n, 1024):  # bounded fp32 scratch
+            c1 = min(n, c0 + 1024)
+            k = torch.randn((c1 - c0,) + shape[1:], generator=g, device=dev)
+            if cfg.new_key_outliers:
+                m = torch.rand((c1 - c0,) + shape[1:3] + (1,), generator=g, device=dev)
+                k += (m < cfg.key_outlier_frac).float() * (cfg.key_outlier_mag * u_dev)
+            kn[c0:c1] = k.to(torch.bfloat16)
+            vn[c0:c1] = torch.randn((c1 - c0,) + shape[1:], generator=g, device=dev).to(torch.bfloat16)
+        return kn, vn
+
+    n_fresh = max(args.warmup, 3) + args.steps
+    kn_u, vn_u = draw_new_kv(n_fresh, 1000003 * cfg.seed + rank)
+
     def step(i):
-        j = i % n_inputs
-        run(q_all[j], kn_all[j], vn_all[j])
+        run(q_all[i % n_inputs], kn_u[i % n_fresh], vn_u[i % n_fresh])
 
     # warm-up
     for i in range(max(args.warmup, 3)):
@@ -323,10 +352,11 @@ def main():
     if binding.lf_get_status(h) != binding.LF_OK:
         raise RuntimeError(f"device status bits {binding.lf_status_bits(h)} after warm-up")
 
-    # The timed steps are replayed from a captured CUDA graph (one kernel
-    # node per step, inputs cycled), so the host's launch path is not timed.
+    # By default every timed step is launched from Python (the host runs
+    # ahead of the ~0.2 ms kernels, so launches are not on the critical path);
+    # --graph replays a captured CUDA graph instead.
     graph, glen = None, 0
-    if not args.no_graph:
+    if args.graph and not args.no_graph:
         glen = max(d for d in range(1, min(args.steps, n_inputs) + 1) if args.steps % d == 0)
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
@@ -375,8 +405,10 @@ def main():
     e2e = None
     if not args.no_e2e:
         hq = torch.from_numpy(np.stack([x[0] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
-        hk = torch.from_numpy(np.stack([x[1] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
-        hv = torch.from_numpy(np.stack([x[2] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        ek, evv = draw_new_kv(args.e2e_steps + 3, 1000003 * cfg.seed + 7919 + rank)
+        hk = ek.cpu().pin_memory()
+        hv = evv.cpu().pin_memory()
+        del ek, evv
         NBUF = 2
         cs = torch.cuda.Stream()
         d_in = [(torch.empty_like(q_all[0]), torch.empty_like(kn_all[0]), torch.empty_like(vn_all[0]))
@@ -399,11 +431,12 @@ def main():
 
         def e2e_step(i):
             b = i % NBUF
-            j = i % n_inputs
+            j = i % n_inputs  # the query set
+            jn = i % hk.shape[0]  # the step's own new token
             if len(pending) == NBUF:  # buffer b is free once its last step's result is read
                 consume()
             with torch.cuda.stream(cs):
-                for dst, src in zip(d_in[b], (hq[j], hk[j], hv[j])):
+                for dst, src in zip(d_in[b], (hq[j], hk[jn], hv[jn])):
                     dst.copy_(src, non_blocking=True)
                 ev_h2d[b].record(cs)
             stream.wait_event(ev_h2d[b])
@@ -427,7 +460,7 @@ def main():
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(cs)
         for i in range(n_e2e):
-            e2e_step(i)
+            e2e_step(3 + i)  # after the 3 warm-up steps' tokens
         a1.record(cs)
         while pending:
             consume()
@@ -492,7 +525,9 @@ def main():
             "l2": "inputs larger than L2: each step reads the 1 GiB K/V cache (L2 is 126 MB)",
             "tokens_per_s": value * cfg.batch,
             "us_per_step_per_layer": ms_per_step * 1e3,
-            "inputs_cycled": n_inputs,
+            "inputs": (f"new K/V drawn per step on the device ({n_fresh} distinct), queries "
+                       f"cycling {n_inputs} seeded sets" if not glen else
+                       f"graph of {glen} steps: its new tokens repeat every {glen} steps"),
             "launch": (f"CUDA graph of {glen} steps replayed" if glen else "one launch per step from Python"),
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
