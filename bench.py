@@ -6,9 +6,10 @@
 One step = one call of lf_decode_step: attention + score + eviction for a
 whole batch, one kernel launch.  Default workload (the throughput point):
 batch 64, 32 query / 8 KV heads, head_dim 128, bf16 cache, budget 4096,
-sink 4, window 128, full cache, 256 distinct synthetic inputs cycled.  The
-1 GiB KV cache read per step is far larger than L2, so no L2 flush is
-needed between steps.
+sink 4, window 128, full cache.  Every step's new token is distinct (drawn
+on the device); the queries cycle through 256 seeded sets.  The 1 GiB KV
+cache read per step is far larger than L2, so no L2 flush is needed between
+steps.  At least 3 warm-up steps run, whatever --warmup says.
 
 Rank 0 prints ONE JSON line.  Under torchrun each rank runs its own batch
 (weak scaling, no collective on the data path); time is the max over ranks.
@@ -339,14 +340,15 @@ def main():
             vn[c0:c1] = torch.randn((c1 - c0,) + shape[1:], generator=g, device=dev).to(torch.bfloat16)
         return kn, vn
 
-    n_fresh = max(args.warmup, 3) + args.steps
+    warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    n_fresh = warmup + args.steps
     kn_u, vn_u = draw_new_kv(n_fresh, 1000003 * cfg.seed + rank)
 
     def step(i):
         run(q_all[i % n_inputs], kn_u[i % n_fresh], vn_u[i % n_fresh])
 
     # warm-up
-    for i in range(max(args.warmup, 3)):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
     if binding.lf_get_status(h) != binding.LF_OK:
@@ -364,7 +366,7 @@ def main():
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=cap):
             for i in range(glen):
-                step(args.warmup + i)
+                step(warmup + i)
         binding.lf_set_stream(h, stream)
         graph.replay()  # one untimed replay
         torch.cuda.synchronize()
@@ -383,7 +385,7 @@ def main():
             graph.replay()
     else:
         for i in range(args.steps):
-            step(args.warmup + i)
+            step(warmup + i)
     e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize()
@@ -505,7 +507,7 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {
             "workload": workload, "batch": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv,
