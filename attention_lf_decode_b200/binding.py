@@ -29,8 +29,8 @@ LF_SCORE_ALPHA_L1V = 1
 
 EXPORTS = ("lf_init", "lf_set_stream", "lf_prefill_cache", "lf_decode_step",
            "lf_decode_attention", "lf_decode_step_ragged", "lf_decode_attention_ragged",
-           "lf_prefill_cache_fp8", "lf_decode_step_fp8", "lf_decode_attention_fp8", "lf_set_split", "lf_get_split", "lf_set_score",
-           "lf_get_score", "lf_get_status",
+           "lf_prefill_cache_fp8", "lf_decode_step_fp8", "lf_decode_attention_fp8",
+           "lf_set_split", "lf_get_split", "lf_set_score", "lf_get_score", "lf_get_status",
            "lf_status_bits", "lf_destroy", "lf_strerror", "lf_version",
            "lf_decode_step_noalloc")
 
@@ -98,8 +98,9 @@ def _check(code: int, what: str) -> int:
     return code
 
 
-def _ptr(t, dtype, shape, name):
-    """Data pointer of a contiguous CUDA tensor of the given dtype/shape."""
+def _ptr(t, dtype, shape, name, device: Optional[int] = None):
+    """Data pointer of a contiguous CUDA tensor of the given dtype/shape (on
+    CUDA device ``device`` when it is given)."""
     import torch
     if t is None:
         return None
@@ -107,6 +108,8 @@ def _ptr(t, dtype, shape, name):
         raise TypeError(f"{name} must be a torch tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device.index != device:
+        raise ValueError(f"{name} is on cuda:{t.device.index}, expected cuda:{device}")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -116,12 +119,18 @@ def _ptr(t, dtype, shape, name):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _hptr(h, t, dtype, shape, name):
+    """_ptr for a call on handle h: the tensor must be on the handle's device."""
+    return _ptr(t, dtype, shape, name, h.device)
+
+
 class Handle:
     """An ``lf_handle`` plus the shape it was created for."""
 
-    def __init__(self, ptr: ctypes.c_void_p, B, Hq, Hkv, D, max_budget):
+    def __init__(self, ptr: ctypes.c_void_p, B, Hq, Hkv, D, max_budget, device: int):
         self.ptr = ptr
         self.B, self.Hq, self.Hkv, self.D, self.max_budget = B, Hq, Hkv, D, max_budget
+        self.device = device  # the CUDA device index the handle was made on
 
     def __del__(self):
         try:
@@ -138,7 +147,7 @@ def lf_init(B: int, Hq: int, Hkv: int, D: int, max_budget: int, stream=None) -> 
     lib = load_library()
     h = ctypes.c_void_p()
     _check(lib.lf_init(ctypes.byref(h), B, Hq, Hkv, D, max_budget, _stream_ptr(stream)), "lf_init")
-    return Handle(h, B, Hq, Hkv, D, max_budget)
+    return Handle(h, B, Hq, Hkv, D, max_budget, torch.cuda.current_device())
 
 
 def _stream_ptr(stream):
@@ -175,11 +184,12 @@ def lf_prefill_cache(h: Handle, k, v, n: int, kcache, vcache, pos, budget: int) 
     import torch
     bf = torch.bfloat16
     cshape = (h.B, h.Hkv, budget, h.D)
-    kp = _ptr(k, bf, (h.B, h.Hkv, n, h.D), "k") if n > 0 else None
-    vp = _ptr(v, bf, (h.B, h.Hkv, n, h.D), "v") if n > 0 else None
+    kp = _hptr(h, k, bf, (h.B, h.Hkv, n, h.D), "k") if n > 0 else None
+    vp = _hptr(h, v, bf, (h.B, h.Hkv, n, h.D), "v") if n > 0 else None
     _check(load_library().lf_prefill_cache(
-        h.ptr, kp, vp, n, _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget), "lf_prefill_cache")
+        h.ptr, kp, vp, n, _hptr(h, kcache, bf, cshape, "kcache"),
+        _hptr(h, vcache, bf, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget), "lf_prefill_cache")
 
 
 def lf_decode_step(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int, sink: int,
@@ -188,12 +198,13 @@ def lf_decode_step(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
     bf = torch.bfloat16
     cshape = (h.B, h.Hkv, budget, h.D)
     _check(load_library().lf_decode_step(
-        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
-        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
-        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget, sink, window,
-        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out"),
-        _ptr(evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step")
+        h.ptr, _hptr(h, q, bf, (h.B, h.Hq, h.D), "q"),
+        _hptr(h, k_new, bf, (h.B, h.Hkv, h.D), "k_new"),
+        _hptr(h, v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _hptr(h, kcache, bf, cshape, "kcache"), _hptr(h, vcache, bf, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget, sink, window,
+        _hptr(h, out, torch.float32, (h.B, h.Hq, h.D), "out"),
+        _hptr(h, evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step")
 
 
 def lf_decode_attention(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int, out) -> None:
@@ -201,11 +212,12 @@ def lf_decode_attention(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget:
     bf = torch.bfloat16
     cshape = (h.B, h.Hkv, budget, h.D)
     _check(load_library().lf_decode_attention(
-        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
-        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
-        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
-        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention")
+        h.ptr, _hptr(h, q, bf, (h.B, h.Hq, h.D), "q"),
+        _hptr(h, k_new, bf, (h.B, h.Hkv, h.D), "k_new"),
+        _hptr(h, v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _hptr(h, kcache, bf, cshape, "kcache"), _hptr(h, vcache, bf, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        _hptr(h, out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention")
 
 
 def lf_decode_step_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
@@ -216,13 +228,14 @@ def lf_decode_step_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, budge
     bf = torch.bfloat16
     cshape = (h.B, h.Hkv, budget, h.D)
     _check(load_library().lf_decode_step_ragged(
-        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
-        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
-        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
-        _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"), sink, window,
-        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out"),
-        _ptr(evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step_ragged")
+        h.ptr, _hptr(h, q, bf, (h.B, h.Hq, h.D), "q"),
+        _hptr(h, k_new, bf, (h.B, h.Hkv, h.D), "k_new"),
+        _hptr(h, v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _hptr(h, kcache, bf, cshape, "kcache"), _hptr(h, vcache, bf, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        _hptr(h, seq_budget, torch.int32, (h.B,), "seq_budget"), sink, window,
+        _hptr(h, out, torch.float32, (h.B, h.Hq, h.D), "out"),
+        _hptr(h, evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step_ragged")
 
 
 def lf_decode_attention_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
@@ -231,12 +244,13 @@ def lf_decode_attention_ragged(h: Handle, q, k_new, v_new, kcache, vcache, pos, 
     bf = torch.bfloat16
     cshape = (h.B, h.Hkv, budget, h.D)
     _check(load_library().lf_decode_attention_ragged(
-        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
-        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
-        _ptr(kcache, bf, cshape, "kcache"), _ptr(vcache, bf, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
-        _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
-        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention_ragged")
+        h.ptr, _hptr(h, q, bf, (h.B, h.Hq, h.D), "q"),
+        _hptr(h, k_new, bf, (h.B, h.Hkv, h.D), "k_new"),
+        _hptr(h, v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _hptr(h, kcache, bf, cshape, "kcache"), _hptr(h, vcache, bf, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        _hptr(h, seq_budget, torch.int32, (h.B,), "seq_budget"),
+        _hptr(h, out, torch.float32, (h.B, h.Hq, h.D), "out")), "lf_decode_attention_ragged")
 
 
 def lf_prefill_cache_fp8(h: Handle, k, v, n: int, kcache, vcache, pos, budget: int,
@@ -246,11 +260,12 @@ def lf_prefill_cache_fp8(h: Handle, k, v, n: int, kcache, vcache, pos, budget: i
     import torch
     bf, u8 = torch.bfloat16, torch.uint8
     cshape = (h.B, h.Hkv, budget, h.D)
-    kp = _ptr(k, bf, (h.B, h.Hkv, n, h.D), "k") if n > 0 else None
-    vp = _ptr(v, bf, (h.B, h.Hkv, n, h.D), "v") if n > 0 else None
+    kp = _hptr(h, k, bf, (h.B, h.Hkv, n, h.D), "k") if n > 0 else None
+    vp = _hptr(h, v, bf, (h.B, h.Hkv, n, h.D), "v") if n > 0 else None
     _check(load_library().lf_prefill_cache_fp8(
-        h.ptr, kp, vp, n, _ptr(kcache, u8, cshape, "kcache"), _ptr(vcache, u8, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget, k_scale, v_scale),
+        h.ptr, kp, vp, n, _hptr(h, kcache, u8, cshape, "kcache"),
+        _hptr(h, vcache, u8, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget, k_scale, v_scale),
         "lf_prefill_cache_fp8")
 
 
@@ -262,14 +277,16 @@ def lf_decode_step_fp8(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: 
     bf, u8 = torch.bfloat16, torch.uint8
     cshape = (h.B, h.Hkv, budget, h.D)
     _check(load_library().lf_decode_step_fp8(
-        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
-        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
-        _ptr(kcache, u8, cshape, "kcache"), _ptr(vcache, u8, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
-        None if seq_budget is None else _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
+        h.ptr, _hptr(h, q, bf, (h.B, h.Hq, h.D), "q"),
+        _hptr(h, k_new, bf, (h.B, h.Hkv, h.D), "k_new"),
+        _hptr(h, v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _hptr(h, kcache, u8, cshape, "kcache"), _hptr(h, vcache, u8, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        None if seq_budget is None
+        else _hptr(h, seq_budget, torch.int32, (h.B,), "seq_budget"),
         sink, window, k_scale, v_scale,
-        _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out"),
-        _ptr(evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step_fp8")
+        _hptr(h, out, torch.float32, (h.B, h.Hq, h.D), "out"),
+        _hptr(h, evicted_idx, torch.int32, (h.B, h.Hkv), "evicted_idx")), "lf_decode_step_fp8")
 
 
 def lf_decode_attention_fp8(h: Handle, q, k_new, v_new, kcache, vcache, pos, budget: int,
@@ -278,12 +295,14 @@ def lf_decode_attention_fp8(h: Handle, q, k_new, v_new, kcache, vcache, pos, bud
     bf, u8 = torch.bfloat16, torch.uint8
     cshape = (h.B, h.Hkv, budget, h.D)
     _check(load_library().lf_decode_attention_fp8(
-        h.ptr, _ptr(q, bf, (h.B, h.Hq, h.D), "q"),
-        _ptr(k_new, bf, (h.B, h.Hkv, h.D), "k_new"), _ptr(v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
-        _ptr(kcache, u8, cshape, "kcache"), _ptr(vcache, u8, cshape, "vcache"),
-        _ptr(pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
-        None if seq_budget is None else _ptr(seq_budget, torch.int32, (h.B,), "seq_budget"),
-        k_scale, v_scale, _ptr(out, torch.float32, (h.B, h.Hq, h.D), "out")),
+        h.ptr, _hptr(h, q, bf, (h.B, h.Hq, h.D), "q"),
+        _hptr(h, k_new, bf, (h.B, h.Hkv, h.D), "k_new"),
+        _hptr(h, v_new, bf, (h.B, h.Hkv, h.D), "v_new"),
+        _hptr(h, kcache, u8, cshape, "kcache"), _hptr(h, vcache, u8, cshape, "vcache"),
+        _hptr(h, pos, torch.int32, (h.B, h.Hkv, budget), "pos"), budget,
+        None if seq_budget is None
+        else _hptr(h, seq_budget, torch.int32, (h.B,), "seq_budget"),
+        k_scale, v_scale, _hptr(h, out, torch.float32, (h.B, h.Hq, h.D), "out")),
         "lf_decode_attention_fp8")
 
 
@@ -297,13 +316,15 @@ def lf_decode_step_noalloc(q, k_new, v_new, kcache, vcache, pos, budget: int, si
     B, Hq, D = q.shape
     Hkv = kcache.shape[1]
     cshape = (B, Hkv, budget, D)
+    dev = torch.cuda.current_device()  # the call runs on the current device
     _check(load_library().lf_decode_step_noalloc(
-        _ptr(q, bf, (B, Hq, D), "q"), _ptr(k_new, bf, (B, Hkv, D), "k_new"),
-        _ptr(v_new, bf, (B, Hkv, D), "v_new"), _ptr(kcache, bf, cshape, "kcache"),
-        _ptr(vcache, bf, cshape, "vcache"), _ptr(pos, torch.int32, (B, Hkv, budget), "pos"),
+        _ptr(q, bf, (B, Hq, D), "q", dev), _ptr(k_new, bf, (B, Hkv, D), "k_new", dev),
+        _ptr(v_new, bf, (B, Hkv, D), "v_new", dev), _ptr(kcache, bf, cshape, "kcache", dev),
+        _ptr(vcache, bf, cshape, "vcache", dev),
+        _ptr(pos, torch.int32, (B, Hkv, budget), "pos", dev),
         B, Hq, Hkv, D, budget, sink, window,
-        _ptr(out, torch.float32, (B, Hq, D), "out"),
-        _ptr(evicted_idx, torch.int32, (B, Hkv), "evicted_idx"), _stream_ptr(stream)),
+        _ptr(out, torch.float32, (B, Hq, D), "out", dev),
+        _ptr(evicted_idx, torch.int32, (B, Hkv), "evicted_idx", dev), _stream_ptr(stream)),
         "lf_decode_step_noalloc")
 
 

@@ -94,6 +94,12 @@ bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(pt
 
 bool valid_handle(lf_handle h) { return h != nullptr && h->magic == kMagic; }
 
+// calls that plan or enqueue work run on the device the handle was made on
+bool on_handle_device(const lf_ctx* c) {
+  int cur = -1;
+  return cudaGetDevice(&cur) == cudaSuccess && cur == c->device;
+}
+
 // the compiled variants, by [E4M3 storage][kernel mode]
 using PlanFn = cudaError_t (*)(int, int, const lf::PlanIn&, int, Plan*);
 using LaunchFn = cudaError_t (*)(int, int, const lf::Params&, const Plan&, cudaStream_t);
@@ -169,6 +175,7 @@ int run_decode(lf_handle h, const uint16_t* q, const uint16_t* k_new, const uint
                const int32_t* seq_budget = nullptr, bool fp8 = false, float k_scale = 1.f,
                float v_scale = 1.f) {
   if (!valid_handle(h)) return LF_ENOTINIT;
+  if (!on_handle_device(h)) return LF_EINVAL;
   if (fp8 && (!good_scale(k_scale) || !good_scale(v_scale))) return LF_EINVAL;
   if (seq_budget && (!aligned(seq_budget, 4) || !h->grab)) return LF_EINVAL;
   if (!q || !k_new || !v_new || !kcache || !vcache || !pos || !out) return LF_EINVAL;
@@ -320,7 +327,7 @@ int lf_get_score(lf_handle h) {
 
 int lf_get_split(lf_handle h, int budget) {
   if (!valid_handle(h)) return LF_ENOTINIT;
-  if (budget < 1 || budget > h->max_budget) return LF_EINVAL;
+  if (budget < 1 || budget > h->max_budget || !on_handle_device(h)) return LF_EINVAL;
   Plan* pl = nullptr;
   const cudaError_t pe = get_plan(h, budget, false, kernel_mode(h, true), &pl);
   if (pe == cudaErrorInvalidConfiguration) return LF_EINVAL;
@@ -331,6 +338,7 @@ int lf_get_split(lf_handle h, int budget) {
 int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, int n, uint16_t* kcache,
                      uint16_t* vcache, int32_t* pos, int budget) {
   if (!valid_handle(h)) return LF_ENOTINIT;
+  if (!on_handle_device(h)) return LF_EINVAL;
   if (budget < 1 || budget > h->max_budget || n < 0 || n > budget) return LF_EINVAL;
   if (!kcache || !vcache || !pos || (n > 0 && (!k || !v))) return LF_EINVAL;
   if (!aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(pos, 4) ||
@@ -351,6 +359,7 @@ int lf_prefill_cache(lf_handle h, const uint16_t* k, const uint16_t* v, int n, u
 int lf_prefill_cache_fp8(lf_handle h, const uint16_t* k, const uint16_t* v, int n, uint8_t* kcache,
                          uint8_t* vcache, int32_t* pos, int budget, float k_scale, float v_scale) {
   if (!valid_handle(h)) return LF_ENOTINIT;
+  if (!on_handle_device(h)) return LF_EINVAL;
   if (budget < 1 || budget > h->max_budget || n < 0 || n > budget) return LF_EINVAL;
   if (!good_scale(k_scale) || !good_scale(v_scale)) return LF_EINVAL;
   if (!kcache || !vcache || !pos || (n > 0 && (!k || !v))) return LF_EINVAL;

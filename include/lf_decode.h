@@ -47,6 +47,11 @@
  *   - Calls are asynchronous on the stream given to lf_init (or
  *     lf_set_stream); arguments are checked on the host before anything is
  *     enqueued.  A failed check enqueues nothing.
+ *   - A handle belongs to the device that was current at lf_init.  Calls
+ *     that plan or enqueue work with it (prefill, decode, lf_get_split)
+ *     return LF_EINVAL, enqueueing nothing, when another device is
+ *     current.  Every tensor must be memory of that device; this is not
+ *     checked (the pointer's device is not queried on the hot path).
  *   - Return codes (never exceptions): LF_OK, or one of the negative
  *     LF_E* codes below; lf_strerror names them.
  */

@@ -84,3 +84,25 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
             if f.endswith(".py"):
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle", src, re.M), f
+
+
+def test_binding_rejects_a_tensor_on_another_device():
+    """A call on a handle checks that every tensor is on the handle's device
+    before anything reaches the library (tensors faked on the CPU)."""
+    import torch
+
+    class OnCuda1(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+        @property
+        def device(self):
+            return torch.device("cuda", 1)
+
+    t = torch.Tensor._make_subclass(OnCuda1, torch.zeros(4, dtype=torch.bfloat16))
+    h = binding.Handle(None, 1, 1, 1, 64, 4, device=0)
+    with pytest.raises(ValueError, match="cuda:1, expected cuda:0"):
+        binding._hptr(h, t, torch.bfloat16, (4,), "q")
+    h1 = binding.Handle(None, 1, 1, 1, 64, 4, device=1)
+    assert binding._hptr(h1, t, torch.bfloat16, (4,), "q").value == t.data_ptr()
