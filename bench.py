@@ -400,10 +400,12 @@ def main():
     # End to end, through the public call: every step copies its inputs from
     # pinned host memory to the device, runs lf_decode_step, copies out and
     # evicted_idx back to pinned host memory, and the host reads that result.
-    # The steps are pipelined two deep: copies run on a second stream into
-    # double-buffered device and host buffers, so step i's copies overlap
-    # steps i - 1 and i + 1, and the host reads step i's result once step
-    # i + 2 has been enqueued.
+    # The steps are pipelined two deep into double-buffered device and host
+    # buffers.  Host-to-device copies run on one copy stream and
+    # device-to-host copies on another, so step i + 1's inputs arrive while
+    # step i computes, and step i's results return while step i + 1
+    # computes.  The host reads step i's result before it enqueues step
+    # i + 2, which reuses step i's buffers (that read also orders the reuse).
     e2e = None
     if not args.no_e2e:
         hq = torch.from_numpy(np.stack([x[0] for x in inputs]).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -412,7 +414,8 @@ def main():
         hv = evv.cpu().pin_memory()
         del ek, evv
         NBUF = 2
-        cs = torch.cuda.Stream()
+        cs_in = torch.cuda.Stream()   # host-to-device copies
+        cs_out = torch.cuda.Stream()  # device-to-host copies
         d_in = [(torch.empty_like(q_all[0]), torch.empty_like(kn_all[0]), torch.empty_like(vn_all[0]))
                 for _ in range(NBUF)]
         d_out = [out] + [torch.empty_like(out) for _ in range(NBUF - 1)]
@@ -437,18 +440,18 @@ def main():
             jn = i % hk.shape[0]  # the step's own new token
             if len(pending) == NBUF:  # buffer b is free once its last step's result is read
                 consume()
-            with torch.cuda.stream(cs):
+            with torch.cuda.stream(cs_in):
                 for dst, src in zip(d_in[b], (hq[j], hk[jn], hv[jn])):
                     dst.copy_(src, non_blocking=True)
-                ev_h2d[b].record(cs)
+                ev_h2d[b].record(cs_in)
             stream.wait_event(ev_h2d[b])
             run(*d_in[b], out=d_out[b], ev=d_ev[b])
             ev_k[b].record(stream)
-            with torch.cuda.stream(cs):
-                cs.wait_event(ev_k[b])
+            with torch.cuda.stream(cs_out):
+                cs_out.wait_event(ev_k[b])
                 h_out[b].copy_(d_out[b], non_blocking=True)
                 h_ev[b].copy_(d_ev[b], non_blocking=True)
-                ev_d2h[b].record(cs)
+                ev_d2h[b].record(cs_out)
             pending.append(b)
 
         for i in range(3):
@@ -460,10 +463,10 @@ def main():
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(cs)
+        a0.record(cs_in)  # before the first step's input copies
         for i in range(n_e2e):
             e2e_step(3 + i)  # after the 3 warm-up steps' tokens
-        a1.record(cs)
+        a1.record(cs_out)  # after the last step's result copies
         while pending:
             consume()
         a1.synchronize()
@@ -474,9 +477,9 @@ def main():
                "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": ems / n_e2e,
                "note": "per step: pinned H2D of q/k_new/v_new, lf_decode_step, D2H of out and "
-                       "evicted_idx, host read of the result; pipelined two steps deep on a "
-                       "copy stream with double-buffered inputs and outputs; the KV cache "
-                       "stays resident"}
+                       "evicted_idx, host read of the result; pipelined two steps deep "
+                       "(H2D and D2H on two copy streams, double-buffered inputs and "
+                       "outputs); the KV cache stays resident"}
         if binding.lf_get_status(h) != binding.LF_OK:
             raise RuntimeError("device status after e2e")
 
