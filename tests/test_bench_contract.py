@@ -78,11 +78,14 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle"
 
 
-@pytest.mark.parametrize("args", [["--kv", "fp8"], ["--score", "alpha_l1v"]])
+@pytest.mark.parametrize("args", [["--kv", "fp8"], ["--score", "alpha_l1v"],
+                                  ["--config", "ragged"]])
 def test_reference_arm_options(args):
     env = dict(os.environ, OMP_NUM_THREADS="1")
+    if "--config" not in args:
+        args = ["--config", "tiny"] + args
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--config", "tiny", "--steps", "1", "--warmup", "0"] + args,
+                        "--steps", "1", "--warmup", "0"] + args,
                        capture_output=True, text=True, cwd=ROOT, env=env, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     assert json.loads(r.stdout.splitlines()[-1])["value"] > 0
