@@ -47,6 +47,9 @@
  *   - Calls are asynchronous on the stream given to lf_init (or
  *     lf_set_stream); arguments are checked on the host before anything is
  *     enqueued.  A failed check enqueues nothing.
+ *   - A handle is not thread-safe: it caches launch plans and holds the
+ *     status word, so calls on one handle come from one thread at a time.
+ *     Separate handles are independent.
  *   - A handle belongs to the device that was current at lf_init.  Calls
  *     that plan or enqueue work with it (prefill, decode, lf_get_split)
  *     return LF_EINVAL, enqueueing nothing, when another device is
