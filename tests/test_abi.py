@@ -86,23 +86,96 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
                 assert not re.search(r"^\s*(import|from)\s+oracle", src, re.M), f
 
 
-def test_binding_rejects_a_tensor_on_another_device():
-    """A call on a handle checks that every tensor is on the handle's device
-    before anything reaches the library (tensors faked on the CPU)."""
+def _fake_cuda(shape, dtype, index=0):
+    """A CPU tensor that reports itself as living on cuda:<index>; only its
+    metadata is read (the library is never called with it)."""
     import torch
 
-    class OnCuda1(torch.Tensor):
+    class FakeCuda(torch.Tensor):
         @property
         def is_cuda(self):
             return True
 
         @property
         def device(self):
-            return torch.device("cuda", 1)
+            return torch.device("cuda", index)
 
-    t = torch.Tensor._make_subclass(OnCuda1, torch.zeros(4, dtype=torch.bfloat16))
+    return torch.Tensor._make_subclass(FakeCuda, torch.zeros(shape, dtype=dtype))
+
+
+def test_binding_rejects_a_tensor_on_another_device():
+    """A call on a handle checks that every tensor is on the handle's device
+    before anything reaches the library."""
+    import torch
+    t = _fake_cuda((4,), torch.bfloat16, index=1)
     h = binding.Handle(None, 1, 1, 1, 64, 4, device=0)
     with pytest.raises(ValueError, match="cuda:1, expected cuda:0"):
         binding._hptr(h, t, torch.bfloat16, (4,), "q")
     h1 = binding.Handle(None, 1, 1, 1, 64, 4, device=1)
     assert binding._hptr(h1, t, torch.bfloat16, (4,), "q").value == t.data_ptr()
+
+
+def test_every_wrapper_marshals_its_arguments(lib, monkeypatch):
+    """Each Python wrapper calls its C function with as many arguments as the
+    ctypes signature declares, pointers as c_void_p (or None where the header
+    allows NULL); a recording stand-in replaces the library, so no CUDA call
+    is made."""
+    import torch
+    calls = []
+
+    class Recorder:
+        def __getattr__(self, name):
+            real = getattr(lib, name)
+
+            def fn(*args):
+                assert len(args) == len(real.argtypes), (name, len(args), len(real.argtypes))
+                for a, t in zip(args, real.argtypes):
+                    if t is ctypes.c_void_p:
+                        assert a is None or isinstance(a, ctypes.c_void_p), (name, a)
+                calls.append(name)
+                return 2 if name == "lf_get_split" else 0
+            return fn
+
+    monkeypatch.setattr(binding, "_lib", Recorder())
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    mk = _fake_cuda
+    B, Hq, Hkv, D, N, n = 2, 8, 2, 64, 32, 16
+    bf, u8, i32, f32 = torch.bfloat16, torch.uint8, torch.int32, torch.float32
+    h = binding.Handle(ctypes.c_void_p(1), B, Hq, Hkv, D, N, device=0)
+    q, kn, vn = mk((B, Hq, D), bf), mk((B, Hkv, D), bf), mk((B, Hkv, D), bf)
+    kc, vc = mk((B, Hkv, N, D), bf), mk((B, Hkv, N, D), bf)
+    kc8, vc8 = mk((B, Hkv, N, D), u8), mk((B, Hkv, N, D), u8)
+    pos, out, ev = mk((B, Hkv, N), i32), mk((B, Hq, D), f32), mk((B, Hkv), i32)
+    kp, vp, nb = mk((B, Hkv, n, D), bf), mk((B, Hkv, n, D), bf), mk((B,), i32)
+
+    binding.lf_set_stream(h, 0)
+    binding.lf_set_split(h, 2)
+    assert binding.lf_get_split(h, N) == 2
+    binding.lf_set_score(h, binding.LF_SCORE_ALPHA_L1V)
+    binding.lf_get_score(h)
+    binding.lf_prefill_cache(h, kp, vp, n, kc, vc, pos, N)
+    binding.lf_prefill_cache(h, None, None, 0, kc, vc, pos, N)
+    binding.lf_decode_step(h, q, kn, vn, kc, vc, pos, N, 4, 8, out, ev)
+    binding.lf_decode_attention(h, q, kn, vn, kc, vc, pos, N, out)
+    binding.lf_decode_step_ragged(h, q, kn, vn, kc, vc, pos, N, nb, 4, 8, out, ev)
+    binding.lf_decode_attention_ragged(h, q, kn, vn, kc, vc, pos, N, nb, out)
+    binding.lf_prefill_cache_fp8(h, kp, vp, n, kc8, vc8, pos, N, 0.5, 2.0)
+    for seq in (None, nb):
+        binding.lf_decode_step_fp8(h, q, kn, vn, kc8, vc8, pos, N, 4, 8, 0.5, 2.0, out, ev, seq)
+        binding.lf_decode_attention_fp8(h, q, kn, vn, kc8, vc8, pos, N, 0.5, 2.0, out, seq)
+    binding.lf_decode_step_noalloc(q, kn, vn, kc, vc, pos, N, 4, 8, out, ev, stream=0)
+    assert binding.lf_get_status(h) == binding.LF_OK
+    binding.lf_status_bits(h)
+    binding.lf_destroy(h)
+    assert h.ptr is None
+    assert set(calls) >= set(binding.EXPORTS) - {"lf_init", "lf_strerror", "lf_version"}
+
+    # a wrongly shaped or typed tensor is refused before the library is called
+    n_calls = len(calls)
+    h = binding.Handle(ctypes.c_void_p(1), B, Hq, Hkv, D, N, device=0)
+    with pytest.raises(ValueError, match="shape"):
+        binding.lf_decode_step(h, q, kn, vn, kc, vc, pos, N + 1, 4, 8, out, ev)
+    with pytest.raises(TypeError, match="uint8"):
+        binding.lf_decode_step_fp8(h, q, kn, vn, kc, vc, pos, N, 4, 8, 1.0, 1.0, out, ev)
+    assert len(calls) == n_calls
+    h.ptr = None
