@@ -98,21 +98,29 @@ def _check(code: int, what: str) -> int:
     return code
 
 
+_Tensor = None  # torch.Tensor, looked up on first use
+
+
 def _ptr(t, dtype, shape, name, device: Optional[int] = None):
     """Data pointer of a contiguous CUDA tensor of the given dtype/shape (on
-    CUDA device ``device`` when it is given)."""
-    import torch
+    CUDA device ``device`` when it is given).  Runs for every tensor of every
+    call, so it keeps to cheap attribute reads (no torch.device objects, no
+    tuple copies)."""
+    global _Tensor
     if t is None:
         return None
-    if not isinstance(t, torch.Tensor):
+    if _Tensor is None:
+        import torch
+        _Tensor = torch.Tensor
+    if not isinstance(t, _Tensor):
         raise TypeError(f"{name} must be a torch tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if device is not None and t.device.index != device:
-        raise ValueError(f"{name} is on cuda:{t.device.index}, expected cuda:{device}")
-    if t.dtype != dtype:
+    if device is not None and t.get_device() != device:
+        raise ValueError(f"{name} is on cuda:{t.get_device()}, expected cuda:{device}")
+    if t.dtype is not dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")

@@ -100,6 +100,9 @@ def _fake_cuda(shape, dtype, index=0):
         def device(self):
             return torch.device("cuda", index)
 
+        def get_device(self):
+            return index
+
     return torch.Tensor._make_subclass(FakeCuda, torch.zeros(shape, dtype=dtype))
 
 
