@@ -10,7 +10,6 @@
 * the step: the scalar brute force on the dequantised cache, torch SDPA on
   the dequantised cache plus the exact new token, and the new token's codes.
 """
-import math
 
 import numpy as np
 import pytest
