@@ -20,6 +20,10 @@ MUTANTS = {
                           "cand = (j >= sink) & (pos <= t - window)"),
     "sink_off_by_one": ("cand = (j >= sink) & (pos < t - window)",
                         "cand = (j > sink) & (pos < t - window)"),
+    "sink_by_position": ("cand = (j >= sink) & (pos < t - window)",
+                         "cand = (pos >= sink) & (pos < t - window)"),
+    "window_by_slot": ("cand = (j >= sink) & (pos < t - window)",
+                       "cand = (j >= sink) & (j < N - window)"),
     "new_token_not_in_denominator": ("l = e.sum(axis=1) + e_new", "l = e.sum(axis=1) + 0 * e_new"),
     "new_token_not_in_max": ("m = np.maximum(s.max(axis=1), s_new)", "m = s.max(axis=1)"),
     "scale_1_over_d": ("scale = 1.0 / math.sqrt(D)", "scale = 1.0 / D"),
